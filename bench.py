@@ -1,0 +1,397 @@
+#!/usr/bin/env python
+"""Benchmark of the mHC forward hot path on B200: one step = mhc_pre + mhc_post
+over T=8192 tokens, n=4 streams, C=4096, bf16 (the LLM-scale sublayer).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  Under torchrun (N > 1) every rank processes
+its own batch of T tokens (weak scaling; the tokens are independent, so no
+collective is on the data path) and the step time is the maximum over ranks.
+
+* value      tokens/s of the whole job, inputs resident in HBM, device-timed
+             with CUDA events over exactly K steps (barrier + synchronize on
+             both sides).  Inputs (X 256 MiB, F_out 64 MiB) exceed the 126 MB
+             L2, so no flush is needed between steps.
+* e2e        the same metric through the public API with pinned HOST buffers:
+             every step copies X and F_out host->device and x_in, the
+             coefficients and X_next device->host.
+* roofline   the dominant kernel's algorithmic bytes per launch / its mean
+             CUDA-event duration inside the timed region, against the measured
+             HBM copy bandwidth.
+* cpu_baseline  the fp64 oracle on a bounded sample of tokens (rank 0, N = 1).
+* --impl reference  runs the oracle (the reference arm of this method): same
+             metric and workload, each step a bounded sample of tokens.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = dict(T=8192, n=4, C=4096, dtype="bf16", seed=1)
+METRIC = "mHC fwd tokens/s at n=4,C=4096; achieved HBM GB/s vs B200 peak"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def algorithmic_bytes(T: int, n: int, C: int, es: int = 2) -> dict:
+    """Bytes each kernel must move per launch (Roofline)."""
+    P = n * n + 2 * n
+    pre = T * (n * C * es + C * es + (2 * n + n * n) * 4) + n * C * P * es + P * 4
+    post = T * (n * C * es + C * es + (n + n * n) * 4 + n * C * es)
+    return {"mhc_pre": pre, "mhc_post": post}
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s)"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampling (200 ms) of SM clocks and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu)], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self._t:
+            self._t.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- dist
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Maximum of a per-rank scalar over all ranks (identity when world == 1)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# -------------------------------------------------------------- oracle leg
+def oracle_sample_rate(inp: dict, seconds: float, max_tokens: int):
+    """Time the fp64 oracle (as it stands) on a bounded sample of the workload's
+    tokens; returns (tokens/s, tokens, threads)."""
+    import oracle
+    oracle.lib()
+    T = inp["T"]
+    probe = min(8, T)
+    t0 = time.perf_counter()
+    oracle.mhc_forward(inp["X"][:probe], inp["F"][:probe], inp["phi"], inp["alpha"], inp["b"],
+                       inp["t_iters"], inp["eps"])
+    per_tok = (time.perf_counter() - t0) / probe
+    S = int(max(1, min(max_tokens, T, seconds / max(per_tok, 1e-9))))
+    t0 = time.perf_counter()
+    oracle.mhc_forward(inp["X"][:S], inp["F"][:S], inp["phi"], inp["alpha"], inp["b"],
+                       inp["t_iters"], inp["eps"])
+    dt = time.perf_counter() - t0
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return S / dt, S, threads
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 oracle, timed on the host cores."""
+    if rank != 0:
+        return
+    import synth
+    import oracle
+    inp = synth.mhc_inputs(**WORKLOAD)
+    oracle.lib()
+    T = inp["T"]
+    # size each step so the whole run stays within about two minutes
+    t0 = time.perf_counter()
+    oracle.mhc_forward(inp["X"][:4], inp["F"][:4], inp["phi"], inp["alpha"], inp["b"])
+    per_tok = (time.perf_counter() - t0) / 4
+    S = int(max(1, min(T, 120.0 / max(per_tok, 1e-9) / max(1, args.steps + args.warmup))))
+    for w in range(args.warmup):
+        oracle.mhc_forward(inp["X"][:S], inp["F"][:S], inp["phi"], inp["alpha"], inp["b"])
+    t0 = time.perf_counter()
+    for k in range(args.steps):
+        lo = (k * S) % max(1, T - S + 1)
+        oracle.mhc_forward(inp["X"][lo:lo + S], inp["F"][lo:lo + S], inp["phi"], inp["alpha"], inp["b"])
+    dt = time.perf_counter() - t0
+    value = S * args.steps / dt
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    sample = f"{S} tokens per step of the T=8192, n=4, C=4096 bf16 workload (inputs widened to fp64)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, synth.mhc_inputs)",
+        "config": config_dict(args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(N: int) -> dict:
+    return {"workload": "mHC forward sublayer (mhc_pre + mhc_post), T=8192 tokens per GPU, "
+                        "n=4, C=4096, bf16 state, fp32 coefficients, Sinkhorn 20 iterations",
+            "T_per_gpu": WORKLOAD["T"], "n": WORKLOAD["n"], "C": WORKLOAD["C"], "t_iters": 20,
+            "global_tokens": WORKLOAD["T"] * N, "parallelism": f"dp{N} (independent token batches)",
+            "l2": "no flush: inputs larger than L2 (X 256 MiB, F_out 64 MiB, X_next 256 MiB vs 126 MB L2)"}
+
+
+# ------------------------------------------------------------------ ours
+def run_ours(args, world, rank, local):
+    import torch
+    import torch.distributed as dist
+    import synth
+    import stream_residual_connections_b200 as M
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    inp = synth.mhc_inputs(**WORKLOAD)
+    T, n, C = inp["T"], inp["n"], inp["C"]
+
+    def to_dev(a):
+        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16) \
+            if a.dtype == np.uint16 else torch.from_numpy(a)
+        return t.to(device)
+
+    X, F, phi = to_dev(inp["X"]), to_dev(inp["F"]), to_dev(inp["phi"])
+    b = torch.from_numpy(inp["b"]).to(device)
+    alpha = inp["alpha"]
+    x_in = torch.empty((T, C), dtype=torch.bfloat16, device=device)
+    Hp = torch.empty((T, n), dtype=torch.float32, device=device)
+    Ho = torch.empty((T, n), dtype=torch.float32, device=device)
+    Hr = torch.empty((T, n, n), dtype=torch.float32, device=device)
+    Xn = torch.empty_like(X)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        M.mhc_pre(X, phi, alpha, b, 20, 1e-6, x_in=x_in, H_pre=Hp, H_post=Ho, H_res=Hr, stream=stream)
+        M.mhc_post(X, F, Ho, Hr, X_next=Xn, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+
+    # --- timed region: K steps, per-kernel events on the launching stream
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    clocks = ClockSampler(device.index if world == 1 else local)
+    if not args.profile:
+        clocks.start()
+    time.sleep(0.3 if K >= 100 else 0.0)
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for k in range(K):
+        ev[k][0].record(stream)
+        M.mhc_pre(X, phi, alpha, b, 20, 1e-6, x_in=x_in, H_pre=Hp, H_post=Ho, H_res=Hr, stream=stream)
+        ev[k][1].record(stream)
+        M.mhc_post(X, F, Ho, Hr, X_next=Xn, stream=stream)
+        ev[k][2].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    clk = clocks.stop()
+    ms_local = start.elapsed_time(end)
+    ms = max_over_ranks(ms_local, world, device)
+    pre_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
+    post_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    ms_per_step = ms / K
+    value = world * T * K / (ms / 1e3)
+
+    if args.profile:
+        if rank == 0:
+            print(json.dumps({"profile": True, "T": T, "steps": K, "ms_per_step": ms_per_step,
+                              "mhc_pre_ms": pre_ms, "mhc_post_ms": post_ms}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    # --- end to end through the public API with host buffers
+    Ke = max(1, min(K, args.e2e_steps))
+    Xh = torch.from_numpy(np.ascontiguousarray(inp["X"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+    Fh = torch.from_numpy(np.ascontiguousarray(inp["F"]).view(np.int16)).view(torch.bfloat16).pin_memory()
+    outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (x_in, Hp, Ho, Hr, Xn)]
+    h2d = Xh.numel() * 2 + Fh.numel() * 2
+    d2h = sum(t.numel() * t.element_size() for t in outs_h)
+
+    def e2e_step():
+        X.copy_(Xh, non_blocking=True)
+        F.copy_(Fh, non_blocking=True)
+        step()
+        for h, d in zip(outs_h, (x_in, Hp, Ho, Hr, Xn)):
+            h.copy_(d, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(Ke):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    e2e_ms = max_over_ranks(s2.elapsed_time(e2), world, device)
+    e2e_value = world * T * Ke / (e2e_ms / 1e3)
+
+    # --- roofline of the dominant kernel
+    peak, peak_src = measured_peak()
+    ab = algorithmic_bytes(T, n, C)
+    kern = {"mhc_pre": pre_ms, "mhc_post": post_ms}
+    kern_rows = {}
+    for name, kms in kern.items():
+        gbs = ab[name] / (kms / 1e3) / 1e9
+        kern_rows[name] = {"ms": kms, "algorithmic_bytes": ab[name], "achieved_gbs": gbs,
+                           "frac": gbs / peak, "share": kms / (pre_ms + post_ms)}
+    dom = max(kern, key=kern.get)
+    traffic = TRAFFIC.get(dom)
+    roof = {"bound": "hbm", "achieved": kern_rows[dom]["achieved_gbs"], "peak": peak, "unit": "GB/s",
+            "frac": kern_rows[dom]["frac"], "traffic": traffic, "kernel": dom,
+            "peak_source": peak_src}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, S, threads = oracle_sample_rate(inp, seconds=args.cpu_seconds, max_tokens=T)
+        cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"first {S} tokens of the same T=8192, n=4, C=4096 workload, fp64 oracle "
+                         f"(mhc_pre + mhc_post), OpenMP over tokens"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded numpy PCG64, synth.mhc_inputs)",
+            "config": config_dict(world),
+            "gpu_launches": 2 * K,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": Ke},
+            "roofline": roof,
+            "kernels": kern_rows,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the current
+# kernels on this workload (profiles/*.txt); None until captured for the
+# kernel version in the tree.
+TRAFFIC = {}
+
+
+def main(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--profile", action="store_true",
+                   help="only warm-up + timed kernel launches (for ncu); no e2e, clocks or oracle")
+    p.add_argument("--tokens", type=int, default=None, help="override T (profiling of small cases)")
+    args = p.parse_args(argv)
+    if args.tokens:
+        WORKLOAD["T"] = args.tokens
+    world, rank, local = dist_env()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return 0
+    run_ours(args, world, rank, local)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,113 @@
+/*
+ * mhc.h -- C ABI of the B200 (sm_100a) residual-stream mixing library (libmhc.so).
+ *
+ * The library computes the per-token residual-stream mixing of one
+ * Transformer sublayer as defined by
+ *   [mHC]  "mHC: Manifold-Constrained Hyper-Connections" (paper notes page):
+ *          section 3 Eq.(3) (single-layer update), section 4.2 Eq.(7)-(9)
+ *          (coefficients), section 4.3.1 Eq.(10)-(19) and the F_pre /
+ *          F_post,res apply kernels;
+ *   [xHC]  "xHC: Expanded Hyper-Connections" (summary page): sections
+ *          "temporal feature augmentation", "sparse residual stream
+ *          architecture", "parameterisation"; and the xHC project page's
+ *          "default xHC configuration" table.
+ *
+ * Common conventions (every entry point):
+ *  - Pointers are DEVICE pointers owned by the caller unless marked "host".
+ *    The library never allocates device memory and keeps no pointer after a
+ *    call returns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  Argument errors are detected on the host before any
+ *    launch and return MHC_ERR_INVALID_ARG or MHC_ERR_UNSUPPORTED with nothing
+ *    enqueued; a launch failure returns MHC_ERR_CUDA.  mhc_last_error() gives
+ *    the message of the last failing call on the calling thread.
+ *  - Layouts are row-major and dense.  The multi-stream state of T tokens is
+ *    X[T][n][C] (each token's n*C row contiguous; vec(X_t) index = i*C + c).
+ *  - dtype: MHC_BF16 (bfloat16 storage) or MHC_F32.  All arithmetic is fp32
+ *    with fp32 accumulation; a bf16 output is rounded once, to nearest even,
+ *    when stored.  Coefficients (H_*) are always fp32.
+ *  - Alignment: every array pointer 16-byte aligned; C a multiple of 8.
+ *  - Sizes: 1 <= n <= 8; T >= 0 (T == 0 enqueues nothing and returns MHC_OK);
+ *    0 <= t_iters <= 1000; eps >= 0.
+ */
+#ifndef MHC_H
+#define MHC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MHC_OK = 0,
+    MHC_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, forbidden aliasing */
+    MHC_ERR_UNSUPPORTED = 2,  /* valid but outside what this build implements        */
+    MHC_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed                  */
+    MHC_ERR_TIMEOUT = 4       /* a bounded on-device wait expired (see mhc_sync_status)*/
+} mhc_status;
+
+typedef enum { MHC_F32 = 0, MHC_BF16 = 1 } mhc_dtype;
+
+/* Message of the last failing call on this thread ("" if none).  Never NULL. */
+const char* mhc_last_error(void);
+
+/* Library ABI version (major*100 + minor). */
+int mhc_version(void);
+
+/*
+ * mhc_pre -- the pre half of one mHC sublayer.   [mHC] Eq.(7), (8), (9); the
+ * fused order of Eq.(14)-(19); F_pre := H_pre x_l (section 4.3.1).
+ *
+ * For every token t:
+ *   x = vec(X_t) (length nC); s = sum(x^2); r = sqrt(s/(nC) + eps)
+ *   z = alpha_seg * (x phi) / r + b            (P = n*n + 2n logits)
+ *   H_pre  = sigmoid(z[0:n]);  H_post = 2*sigmoid(z[n:2n])
+ *   H_res  = Sinkhorn-Knopp(z[2n:], row-major n x n): M = exp(z_res); t_iters times
+ *            { normalise every column to sum 1; then every row }
+ *   x_in[c] = sum_i H_pre[i] * X_t[i][c]
+ *
+ *   X      [T][n][C], dtype x_dt                       (read)
+ *   phi    [n*C][P],  dtype phi_dt; columns pre n | post n | res n*n (read)
+ *   alpha  HOST float[3] = (alpha_pre, alpha_post, alpha_res)
+ *   b      [P] fp32                                    (read)
+ *   x_in   [T][C], dtype x_dt                          (written)
+ *   H_pre  [T][n] fp32, may be NULL                    (written)
+ *   H_post [T][n] fp32                                 (written)
+ *   H_res  [T][n][n] fp32 (H_res[t][i][j] weights source stream j into i) (written)
+ * Supported (x_dt, phi_dt): (F32, F32), (BF16, BF16), (BF16, F32).
+ * Outputs must not overlap any input.
+ */
+mhc_status mhc_pre(const void* X, mhc_dtype x_dt, const void* phi, mhc_dtype phi_dt,
+                   const float* alpha, const float* b, int64_t T, int n, int C,
+                   int t_iters, float eps, void* x_in, float* H_pre, float* H_post,
+                   float* H_res, void* stream);
+
+/*
+ * mhc_post -- the post half of one mHC sublayer.   [mHC] Eq.(3) and the fused
+ * F_post,res := H_res x_l + H_post^T F kernel of section 4.3.1 (reads (n+1)C
+ * and writes nC elements per token).
+ *
+ *   X_next[t][i][c] = sum_j H_res[t][i][j] * X[t][j][c] + H_post[t][i] * F_out[t][c]
+ *
+ *   X      [T][n][C], dtype dt (read)      F_out [T][C], dtype dt (read)
+ *   H_post [T][n] fp32, H_res [T][n][n] fp32 (read; e.g. from mhc_pre)
+ *   X_next [T][n][C], dtype dt (written).  X_next == X (in place) is allowed;
+ *   any other overlap with an input is rejected.
+ */
+mhc_status mhc_post(const void* X, const void* F_out, mhc_dtype dt, const float* H_post,
+                    const float* H_res, int64_t T, int n, int C, void* X_next, void* stream);
+
+/*
+ * mhc_sync_status -- wait for `stream`, then report and clear the device-side
+ * error word that bounded waits set when they expire: MHC_ERR_TIMEOUT if any
+ * kernel of this library gave up waiting since the last call, else MHC_OK (or
+ * MHC_ERR_CUDA if the stream itself failed).
+ */
+mhc_status mhc_sync_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MHC_H */

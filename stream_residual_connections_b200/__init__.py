@@ -1,0 +1,133 @@
+"""B200 (sm_100a) residual-stream mixing: mHC pre/post, xHC routing / conv +
+Gram-Schmidt / sparse update, and the mHC backward.
+
+This module is a thin binding over the C ABI of ``libmhc.so`` (declared in
+``include/mhc.h``): it checks tensor devices, dtypes and contiguity, allocates
+outputs with torch when the caller does not pass them, and forwards raw
+device pointers and the current CUDA stream.  Every step of the computation
+runs in the library's CUDA kernels; there is no CPU or PyTorch fallback, and
+every call fails loudly (ImportError) if the library has not been built.
+
+Names and arguments follow the C ABI one to one.
+"""
+from __future__ import annotations
+
+import ctypes as ct
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmhc.so")
+
+MHC_OK, MHC_ERR_INVALID_ARG, MHC_ERR_UNSUPPORTED, MHC_ERR_CUDA, MHC_ERR_TIMEOUT = range(5)
+MHC_F32, MHC_BF16 = 0, 1
+_STATUS = {0: "MHC_OK", 1: "MHC_ERR_INVALID_ARG", 2: "MHC_ERR_UNSUPPORTED", 3: "MHC_ERR_CUDA",
+           4: "MHC_ERR_TIMEOUT"}
+
+
+class MhcError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libmhc.so not built ({LIB_PATH}); run "
+                          "`python -m stream_residual_connections_b200.build`")
+    L = ct.CDLL(LIB_PATH)
+    vp, i64, i32, f32 = ct.c_void_p, ct.c_int64, ct.c_int, ct.c_float
+    fp = ct.POINTER(ct.c_float)
+    L.mhc_last_error.restype = ct.c_char_p
+    L.mhc_version.restype = ct.c_int
+    L.mhc_pre.argtypes = [vp, i32, vp, i32, fp, vp, i64, i32, i32, i32, f32, vp, vp, vp, vp, vp]
+    L.mhc_post.argtypes = [vp, vp, i32, vp, vp, i64, i32, i32, vp, vp]
+    L.mhc_sync_status.argtypes = [vp]
+    for name in ("mhc_pre", "mhc_post", "mhc_sync_status"):
+        getattr(L, name).restype = ct.c_int
+    return L
+
+
+_lib = None
+
+
+def native():
+    """The loaded libmhc.so (ctypes.CDLL).  Raises ImportError if it is not built."""
+    global _lib
+    if _lib is None:
+        _lib = _load()
+    return _lib
+
+
+def _check(status: int) -> None:
+    if status != MHC_OK:
+        raise MhcError(status, native().mhc_last_error().decode())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return MHC_BF16
+    if t.dtype == torch.float32:
+        return MHC_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ct.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ct.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _host3(alpha, count=3):
+    vals = [float(v) for v in (alpha.tolist() if hasattr(alpha, "tolist") else alpha)]
+    if len(vals) != count:
+        raise ValueError(f"alpha must have {count} values")
+    return (ct.c_float * count)(*vals)
+
+
+def mhc_pre(X, phi, alpha, b, t_iters: int = 20, eps: float = 1e-6, *, x_in=None, H_pre=None,
+            H_post=None, H_res=None, want_H_pre: bool = True, stream=None):
+    """Pre half of one mHC sublayer (see include/mhc.h).  X [T][n][C], phi [nC][n^2+2n],
+    alpha: 3 host floats, b [n^2+2n] fp32.  Returns (x_in, H_pre, H_post, H_res)."""
+    T, n, C = X.shape
+    dev = X.device
+    if x_in is None:
+        x_in = torch.empty((T, C), dtype=X.dtype, device=dev)
+    if H_pre is None and want_H_pre:
+        H_pre = torch.empty((T, n), dtype=torch.float32, device=dev)
+    if H_post is None:
+        H_post = torch.empty((T, n), dtype=torch.float32, device=dev)
+    if H_res is None:
+        H_res = torch.empty((T, n, n), dtype=torch.float32, device=dev)
+    _check(native().mhc_pre(_ptr(X), _dt(X), _ptr(phi), _dt(phi), _host3(alpha), _ptr(b), T, n, C,
+                       int(t_iters), float(eps), _ptr(x_in), _ptr(H_pre), _ptr(H_post),
+                       _ptr(H_res), _stream(stream)))
+    return x_in, H_pre, H_post, H_res
+
+
+def mhc_post(X, F_out, H_post, H_res, *, X_next=None, stream=None):
+    """Post half: X_next = H_res X + H_post^T F_out.  Pass X_next=X for in place."""
+    T, n, C = X.shape
+    if X_next is None:
+        X_next = torch.empty_like(X)
+    if F_out.dtype != X.dtype:
+        raise TypeError("X and F_out must share a dtype")
+    _check(native().mhc_post(_ptr(X), _ptr(F_out), _dt(X), _ptr(H_post), _ptr(H_res), T, n, C,
+                        _ptr(X_next), _stream(stream)))
+    return X_next
+
+
+def mhc_sync_status(stream=None) -> None:
+    """Wait for the stream; raise MhcError(MHC_ERR_TIMEOUT) if a bounded wait expired."""
+    _check(native().mhc_sync_status(_stream(stream)))

@@ -1,0 +1,160 @@
+// C ABI of libmhc: argument validation, dispatch, error reporting.
+// Declarations and the contract of every entry point are in include/mhc.h.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace mhc {
+
+static thread_local char g_msg[512] = "";
+
+void set_error(const char* fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+}
+
+mhc_status cuda_status(cudaError_t e, const char* what)
+{
+    if (e == cudaSuccess) return MHC_OK;
+    set_error("%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+    return MHC_ERR_CUDA;
+}
+
+mhc_status launch_status(const char* what) { return cuda_status(cudaGetLastError(), what); }
+
+}  // namespace mhc
+
+using namespace mhc;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t dt_size(mhc_dtype d) { return d == MHC_BF16 ? 2 : 4; }
+
+bool valid_dt(mhc_dtype d) { return d == MHC_BF16 || d == MHC_F32; }
+
+struct Range {
+    uintptr_t lo, hi;
+};
+Range range_of(const void* p, size_t bytes)
+{
+    uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return Range{a, a + bytes};
+}
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi && a.hi > a.lo && b.hi > b.lo; }
+
+#define REQUIRE(cond, code, ...)          \
+    do {                                  \
+        if (!(cond)) {                    \
+            set_error(__VA_ARGS__);       \
+            return code;                  \
+        }                                 \
+    } while (0)
+
+#define REQUIRE_PTR(p, name)                                                              \
+    do {                                                                                  \
+        REQUIRE((p) != nullptr, MHC_ERR_INVALID_ARG, "%s: %s is NULL", fn, name);         \
+        REQUIRE(aligned16(p), MHC_ERR_INVALID_ARG, "%s: %s is not 16-byte aligned", fn, name); \
+    } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* mhc_last_error(void) { return g_msg; }
+
+int mhc_version(void) { return 100; }
+
+mhc_status mhc_pre(const void* X, mhc_dtype x_dt, const void* phi, mhc_dtype phi_dt,
+                   const float* alpha, const float* b, int64_t T, int n, int C, int t_iters,
+                   float eps, void* x_in, float* H_pre, float* H_post, float* H_res,
+                   void* stream)
+{
+    const char* fn = "mhc_pre";
+    g_msg[0] = 0;
+    REQUIRE(valid_dt(x_dt) && valid_dt(phi_dt), MHC_ERR_INVALID_ARG, "%s: unknown dtype", fn);
+    REQUIRE(n >= 1 && n <= 8, MHC_ERR_INVALID_ARG, "%s: n=%d outside [1, 8]", fn, n);
+    REQUIRE(C > 0 && C % 8 == 0, MHC_ERR_INVALID_ARG, "%s: C=%d must be a positive multiple of 8", fn, C);
+    REQUIRE(T >= 0, MHC_ERR_INVALID_ARG, "%s: T=%lld < 0", fn, (long long)T);
+    REQUIRE(t_iters >= 0 && t_iters <= 1000, MHC_ERR_INVALID_ARG, "%s: t_iters=%d outside [0, 1000]", fn, t_iters);
+    REQUIRE(eps >= 0.0f, MHC_ERR_INVALID_ARG, "%s: eps < 0", fn);
+    REQUIRE(alpha != nullptr, MHC_ERR_INVALID_ARG, "%s: alpha (host float[3]) is NULL", fn);
+    REQUIRE(!(x_dt == MHC_F32 && phi_dt == MHC_BF16), MHC_ERR_UNSUPPORTED,
+            "%s: fp32 X with bf16 phi is not supported", fn);
+    if (T == 0) return MHC_OK;
+    REQUIRE_PTR(X, "X");
+    REQUIRE_PTR(phi, "phi");
+    REQUIRE_PTR(b, "b");
+    REQUIRE_PTR(x_in, "x_in");
+    REQUIRE_PTR(H_post, "H_post");
+    REQUIRE_PTR(H_res, "H_res");
+    if (H_pre) REQUIRE(aligned16(H_pre), MHC_ERR_INVALID_ARG, "%s: H_pre is not 16-byte aligned", fn);
+    const int P = n * n + 2 * n;
+    const size_t es = dt_size(x_dt);
+    const Range rX = range_of(X, size_t(T) * n * C * es), rphi = range_of(phi, size_t(n) * C * P * dt_size(phi_dt)),
+                rb = range_of(b, size_t(P) * 4);
+    const Range outs[4] = {range_of(x_in, size_t(T) * C * es), range_of(H_pre, H_pre ? size_t(T) * n * 4 : 0),
+                           range_of(H_post, size_t(T) * n * 4), range_of(H_res, size_t(T) * n * n * 4)};
+    for (int i = 0; i < 4; ++i) {
+        REQUIRE(!overlap(outs[i], rX) && !overlap(outs[i], rphi) && !overlap(outs[i], rb),
+                MHC_ERR_INVALID_ARG, "%s: an output overlaps an input", fn);
+        for (int j = 0; j < i; ++j)
+            REQUIRE(!overlap(outs[i], outs[j]), MHC_ERR_INVALID_ARG, "%s: outputs overlap", fn);
+    }
+    PreArgs a{X, x_dt, phi, phi_dt, {alpha[0], alpha[1], alpha[2]}, b, T, n, C, t_iters, eps,
+              x_in, H_pre, H_post, H_res};
+    return launch_pre_fma(a, static_cast<cudaStream_t>(stream));
+}
+
+mhc_status mhc_post(const void* X, const void* F_out, mhc_dtype dt, const float* H_post,
+                    const float* H_res, int64_t T, int n, int C, void* X_next, void* stream)
+{
+    const char* fn = "mhc_post";
+    g_msg[0] = 0;
+    REQUIRE(valid_dt(dt), MHC_ERR_INVALID_ARG, "%s: unknown dtype", fn);
+    REQUIRE(n >= 1 && n <= 8, MHC_ERR_INVALID_ARG, "%s: n=%d outside [1, 8]", fn, n);
+    REQUIRE(C > 0 && C % 8 == 0, MHC_ERR_INVALID_ARG, "%s: C=%d must be a positive multiple of 8", fn, C);
+    REQUIRE(T >= 0, MHC_ERR_INVALID_ARG, "%s: T=%lld < 0", fn, (long long)T);
+    if (T == 0) return MHC_OK;
+    REQUIRE_PTR(X, "X");
+    REQUIRE_PTR(F_out, "F_out");
+    REQUIRE_PTR(H_post, "H_post");
+    REQUIRE_PTR(H_res, "H_res");
+    REQUIRE_PTR(X_next, "X_next");
+    const size_t es = dt_size(dt);
+    const Range rXn = range_of(X_next, size_t(T) * n * C * es);
+    REQUIRE(X_next == X || !overlap(rXn, range_of(X, size_t(T) * n * C * es)), MHC_ERR_INVALID_ARG,
+            "%s: X_next partially overlaps X (only X_next == X is allowed)", fn);
+    REQUIRE(!overlap(rXn, range_of(F_out, size_t(T) * C * es)) &&
+                !overlap(rXn, range_of(H_post, size_t(T) * n * 4)) &&
+                !overlap(rXn, range_of(H_res, size_t(T) * n * n * 4)),
+            MHC_ERR_INVALID_ARG, "%s: X_next overlaps F_out or a coefficient array", fn);
+    return launch_post(X, F_out, dt, H_post, H_res, T, n, C, X_next, static_cast<cudaStream_t>(stream));
+}
+
+mhc_status mhc_sync_status(void* stream)
+{
+    g_msg[0] = 0;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_status(e, "mhc_sync_status");
+    unsigned int flag = 0;
+    e = cudaMemcpyFromSymbol(&flag, g_device_error, sizeof(flag));
+    if (e != cudaSuccess) return cuda_status(e, "mhc_sync_status: read error word");
+    if (flag) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+        if (e != cudaSuccess) return cuda_status(e, "mhc_sync_status: clear error word");
+        set_error("a bounded on-device wait expired (error word 0x%x)", flag);
+        return MHC_ERR_TIMEOUT;
+    }
+    return MHC_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,26 @@
+// Internal launcher interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mhc.h"
+
+namespace mhc {
+
+mhc_status launch_post(const void* X, const void* F, mhc_dtype dt, const float* Hpost,
+                       const float* Hres, int64_t T, int n, int C, void* Xn, cudaStream_t s);
+
+struct PreArgs {
+    const void* X; mhc_dtype x_dt;
+    const void* phi; mhc_dtype phi_dt;
+    float alpha[3];
+    const float* b;
+    int64_t T; int n; int C; int t_iters; float eps;
+    void* x_in; float* H_pre; float* H_post; float* H_res;
+};
+
+// CUDA-core (FMA) projection path: every n, dtype pair and C % 8 == 0.
+mhc_status launch_pre_fma(const PreArgs& a, cudaStream_t s);
+
+}  // namespace mhc

@@ -1,0 +1,5 @@
+// Single translation unit of libmhc: the kernels share a few device globals
+// (the bounded-wait error word and limit), so they are compiled together.
+#include "api.cu"
+#include "mhc_post.cu"
+#include "mhc_pre_fma.cu"

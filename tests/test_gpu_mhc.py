@@ -1,0 +1,153 @@
+"""GPU parity of mhc_pre / mhc_post against the fp64 oracle, through the C ABI.
+
+Small cases span several tiles and a ragged tail and are compared element by
+element; the LLM-scale workload (T=8192, n=4, C=4096, bf16) runs in the
+bench's launch configuration and is compared on sampled tokens."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import stream_residual_connections_b200 as M
+import synth
+from tests.parity import check_coeffs, check_mix, check_rounding, dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(inp, phi_dtype=None):
+    X, F, phi = dev(inp["X"]), dev(inp["F"]), dev(inp["phi"])
+    if phi_dtype == "f32":
+        phi = torch.from_numpy(oracle.widen(inp["phi"]).astype(np.float32)).cuda()
+    b = torch.from_numpy(inp["b"]).cuda()
+    x_in, Hp, Ho, Hr = M.mhc_pre(X, phi, inp["alpha"], b, inp["t_iters"], inp["eps"])
+    Xn = M.mhc_post(X, F, Ho, Hr)
+    torch.cuda.synchronize()
+    return dict(x_in=host(x_in), H_pre=host(Hp), H_post=host(Ho), H_res=host(Hr), X_next=host(Xn))
+
+
+def _compare(inp, got, tokens=None):
+    sel = slice(None) if tokens is None else tokens
+    X = oracle.widen(inp["X"])[sel]
+    F = oracle.widen(inp["F"])[sel]
+    ref = oracle.mhc_forward(X, F, inp["phi"], inp["alpha"], inp["b"], inp["t_iters"], inp["eps"])
+    g = {k: v[sel] for k, v in got.items()}
+    for key in ("H_pre", "H_post", "H_res"):
+        check_coeffs(g[key], ref[key], key)
+    dt = inp["dtype"]
+    absX = np.abs(X).sum(1)
+    miss = check_mix(g["x_in"], ref["x_in"], absX, dt, "x_in")
+    miss += check_mix(g["X_next"], ref["X_next"], absX[:, None, :] + np.abs(F)[:, None, :], dt, "X_next")
+    # rounding-only: the oracle's apply steps fed the GPU's own coefficients
+    ref_in = oracle.mhc_apply_pre(X, g["H_pre"])
+    check_rounding(g["x_in"], ref_in, np.einsum("ti,tic->tc", np.abs(g["H_pre"]), np.abs(X)), dt, "x_in")
+    ref_n = oracle.mhc_post(X, F, g["H_post"], g["H_res"])
+    prods = (np.einsum("tij,tjc->tic", np.abs(g["H_res"]), np.abs(X))
+             + np.abs(g["H_post"])[:, :, None] * np.abs(F)[:, None, :])
+    check_rounding(g["X_next"], ref_n, prods, dt, "X_next")
+    # Sinkhorn output on the GPU: non-negative, rows sum to 1 (last step is T_r)
+    assert (g["H_res"] >= 0).all()
+    np.testing.assert_allclose(g["H_res"].sum(-1), 1.0, atol=2e-6)
+    return miss
+
+
+def test_tiny_fp32_workload():
+    """T=64, n=4, C=256, fp32 throughout (all outputs compared)."""
+    inp = synth.mhc_inputs(**synth.WORKLOADS["mhc_tiny"])
+    _compare(inp, _run(inp))
+
+
+@pytest.mark.parametrize("T,n,C", [(1, 4, 64), (3, 1, 8), (67, 4, 264), (300, 4, 1024),
+                                   (130, 2, 512), (40, 8, 512), (37, 3, 136), (20, 5, 256),
+                                   (9, 6, 96), (11, 7, 64), (257, 4, 4096)])
+def test_bf16_shapes(T, n, C):
+    inp = synth.mhc_inputs(T, n, C, "bf16", seed=100 + T + n + C)
+    _compare(inp, _run(inp))
+
+
+def test_bf16_x_with_fp32_phi():
+    inp = synth.mhc_inputs(70, 4, 512, "bf16", seed=7)
+    inp32 = dict(inp, phi=oracle.widen(inp["phi"]).astype(np.float32))
+    _compare(inp32, _run(inp, phi_dtype="f32"))
+
+
+def test_fp32_shapes_all_n():
+    for n in range(1, 9):
+        inp = synth.mhc_inputs(19, n, 64, "f32", seed=200 + n)
+        _compare(inp, _run(inp))
+
+
+def test_t_iters_zero_and_one():
+    for t in (0, 1, 3):
+        inp = synth.mhc_inputs(25, 4, 128, "f32", seed=300 + t)
+        inp["t_iters"] = t
+        _compare(inp, _run(inp))
+
+
+def test_post_in_place():
+    inp = synth.mhc_inputs(50, 4, 256, "bf16", seed=11)
+    X, F = dev(inp["X"]), dev(inp["F"])
+    b = torch.from_numpy(inp["b"]).cuda()
+    _, _, Ho, Hr = M.mhc_pre(X, dev(inp["phi"]), inp["alpha"], b)
+    ref = M.mhc_post(X, F, Ho, Hr)
+    out = M.mhc_post(X, F, Ho, Hr, X_next=X)
+    torch.cuda.synchronize()
+    assert out.data_ptr() == X.data_ptr()
+    assert torch.equal(ref, X)
+
+
+def test_empty_T_is_a_no_op():
+    X = torch.zeros((0, 4, 64), dtype=torch.bfloat16, device="cuda")
+    phi = torch.zeros((256, 24), dtype=torch.bfloat16, device="cuda")
+    b = torch.zeros(24, device="cuda")
+    x_in, *_ = M.mhc_pre(X, phi, [0.01] * 3, b)
+    assert x_in.shape == (0, 64)
+    M.mhc_post(X, torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda"),
+               torch.zeros((0, 4), device="cuda"), torch.zeros((0, 4, 4), device="cuda"))
+
+
+def test_plain_residual_and_permutation_reduction_bit_exact():
+    """mHC page Eq.(1) vs Eq.(3): alpha = 0 with +-40 biases gives H_res = P_sigma,
+    H_pre = e_2, H_post = 1; x_in = X[2] and X_next[i] = X[sigma(i)] + F, both
+    bit-exact after the single bf16 rounding."""
+    T, n, C = 37, 4, 264
+    inp = synth.mhc_inputs(T, n, C, "bf16", seed=12)
+    sig = [1, 2, 0, 3]
+    b = np.zeros(24, dtype=np.float32)
+    b[:n] = -40.0; b[2] = 40.0
+    res = np.full((n, n), -40.0, dtype=np.float32)
+    for i in range(n):
+        res[i, sig[i]] = 40.0
+    b[2 * n:] = res.reshape(-1)
+    inp["b"] = b
+    inp["alpha"] = np.zeros(3, dtype=np.float32)
+    got = _run(inp)
+    X, F = oracle.widen(inp["X"]), oracle.widen(inp["F"])
+    np.testing.assert_array_equal(got["x_in"], X[:, 2])
+    expect = oracle.widen(synth.f32_to_bf16_bits((X[:, sig] + F[:, None, :]).astype(np.float32)))
+    np.testing.assert_array_equal(got["X_next"], expect)
+    np.testing.assert_allclose(got["H_res"], np.broadcast_to(np.eye(n)[sig], (T, n, n)), atol=1e-30)
+
+
+def test_n1_exact_identity():
+    inp = synth.mhc_inputs(33, 1, 128, "bf16", seed=13)
+    got = _run(inp)
+    assert (got["H_res"] == 1.0).all()
+
+
+def test_llm_workload_sampled_tokens():
+    """T=8192, n=4, C=4096 bf16 (the benchmark's workload and launch configuration):
+    every coefficient and output of 64 sampled tokens, plus properties over all tokens."""
+    inp = synth.mhc_inputs(**synth.WORKLOADS["mhc_llm"])
+    got = _run(inp)
+    rng = np.random.default_rng(0)
+    toks = np.unique(np.concatenate([[0, 1, 8191], rng.choice(8192, 61, replace=False)]))
+    _compare(inp, got, toks)
+    assert np.isfinite(got["X_next"]).all() and np.isfinite(got["x_in"]).all()
+    assert (got["H_res"] >= 0).all()
+    np.testing.assert_allclose(got["H_res"].sum(-1), 1.0, atol=2e-6)
+    np.testing.assert_allclose(got["H_res"].sum(-2), 1.0, atol=1e-3)
+    assert ((got["H_pre"] > 0) & (got["H_pre"] < 1)).all()
+    assert ((got["H_post"] > 0) & (got["H_post"] < 2)).all()
