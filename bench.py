@@ -284,6 +284,21 @@ def run_ours(args, world, rank, local):
     ms_per_step = ms / K
     value = world * T * K / (ms / 1e3)
 
+    # the CUDA-core (FMA) projection path on the same inputs, for comparison
+    fma_ms = None
+    if not args.profile and args.compare_fma:
+        M.mhc_set_path(M.MHC_PATH_FMA)
+        for _ in range(2):
+            M.mhc_pre(X, phi, alpha, b, 20, 1e-6, x_in=x_in, H_pre=Hp, H_post=Ho, H_res=Hr, stream=stream)
+        fs, fe = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fs.record(stream)
+        for _ in range(5):
+            M.mhc_pre(X, phi, alpha, b, 20, 1e-6, x_in=x_in, H_pre=Hp, H_post=Ho, H_res=Hr, stream=stream)
+        fe.record(stream)
+        torch.cuda.synchronize(device)
+        fma_ms = fs.elapsed_time(fe) / 5
+        M.mhc_set_path(M.MHC_PATH_AUTO)
+
     if args.profile:
         if rank == 0:
             print(json.dumps({"profile": True, "T": T, "steps": K, "ms_per_step": ms_per_step,
@@ -354,6 +369,7 @@ def run_ours(args, world, rank, local):
                     "d2h_bytes_per_step": d2h, "steps": Ke},
             "roofline": roof,
             "kernels": kern_rows,
+            "mhc_pre_fma_path_ms": fma_ms,
             "clocks": clk,
             "cpu_baseline": cpu,
         }
@@ -377,6 +393,8 @@ def main(argv=None):
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--compare-fma", type=int, default=1,
+                   help="also time mhc_pre's CUDA-core projection path (5 launches, not in the step)")
     p.add_argument("--profile", action="store_true",
                    help="only warm-up + timed kernel launches (for ncu); no e2e, clocks or oracle")
     p.add_argument("--tokens", type=int, default=None, help="override T (profiling of small cases)")

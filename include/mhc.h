@@ -99,6 +99,31 @@ mhc_status mhc_pre(const void* X, mhc_dtype x_dt, const void* phi, mhc_dtype phi
 mhc_status mhc_post(const void* X, const void* F_out, mhc_dtype dt, const float* H_post,
                     const float* H_res, int64_t T, int n, int C, void* X_next, void* stream);
 
+/* Kernel selection for the projection of mhc_pre. */
+typedef enum {
+    MHC_PATH_AUTO = 0,    /* tensor cores where supported, else CUDA cores (default) */
+    MHC_PATH_FMA = 1,     /* always the CUDA-core (FMA) projection                    */
+    MHC_PATH_TENSOR = 2   /* always tensor cores; calls it cannot serve return        */
+                          /* MHC_ERR_UNSUPPORTED                                       */
+} mhc_path;
+
+/*
+ * mhc_set_path -- process-wide choice of the mhc_pre projection kernel (for
+ * comparisons and tests; both paths compute the same function).  The
+ * tensor-core path (TMA + tcgen05.mma, 8-CTA clusters) serves bf16 X and phi,
+ * n in {2, 3, 4}, C % 512 == 0, 1 <= T < 2^31.
+ */
+mhc_status mhc_set_path(mhc_path path);
+
+/*
+ * mhc_set_wait_limit -- number of polls after which a bounded on-device wait
+ * gives up (default 2^26).  A kernel whose wait expires records it in the
+ * device error word, stops, releases what it holds and returns; its outputs
+ * are then undefined and mhc_sync_status() reports MHC_ERR_TIMEOUT.  Meant
+ * for tests of that failure path; polls >= 1.
+ */
+mhc_status mhc_set_wait_limit(long long polls);
+
 /*
  * mhc_sync_status -- wait for `stream`, then report and clear the device-side
  * error word that bounded waits set when they expire: MHC_ERR_TIMEOUT if any

@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libmhc.so")
 
 MHC_OK, MHC_ERR_INVALID_ARG, MHC_ERR_UNSUPPORTED, MHC_ERR_CUDA, MHC_ERR_TIMEOUT = range(5)
 MHC_F32, MHC_BF16 = 0, 1
+MHC_PATH_AUTO, MHC_PATH_FMA, MHC_PATH_TENSOR = 0, 1, 2
 _STATUS = {0: "MHC_OK", 1: "MHC_ERR_INVALID_ARG", 2: "MHC_ERR_UNSUPPORTED", 3: "MHC_ERR_CUDA",
            4: "MHC_ERR_TIMEOUT"}
 
@@ -44,7 +45,9 @@ def _load():
     L.mhc_pre.argtypes = [vp, i32, vp, i32, fp, vp, i64, i32, i32, i32, f32, vp, vp, vp, vp, vp]
     L.mhc_post.argtypes = [vp, vp, i32, vp, vp, i64, i32, i32, vp, vp]
     L.mhc_sync_status.argtypes = [vp]
-    for name in ("mhc_pre", "mhc_post", "mhc_sync_status"):
+    L.mhc_set_path.argtypes = [i32]
+    L.mhc_set_wait_limit.argtypes = [ct.c_longlong]
+    for name in ("mhc_pre", "mhc_post", "mhc_sync_status", "mhc_set_path", "mhc_set_wait_limit"):
         getattr(L, name).restype = ct.c_int
     return L
 
@@ -131,3 +134,13 @@ def mhc_post(X, F_out, H_post, H_res, *, X_next=None, stream=None):
 def mhc_sync_status(stream=None) -> None:
     """Wait for the stream; raise MhcError(MHC_ERR_TIMEOUT) if a bounded wait expired."""
     _check(native().mhc_sync_status(_stream(stream)))
+
+
+def mhc_set_path(path: int) -> None:
+    """Process-wide mhc_pre projection kernel: MHC_PATH_AUTO / _FMA / _TENSOR."""
+    _check(native().mhc_set_path(int(path)))
+
+
+def mhc_set_wait_limit(polls: int) -> None:
+    """Polls before a bounded on-device wait gives up (tests of the timeout path)."""
+    _check(native().mhc_set_wait_limit(int(polls)))

@@ -28,6 +28,8 @@ mhc_status cuda_status(cudaError_t e, const char* what)
 
 mhc_status launch_status(const char* what) { return cuda_status(cudaGetLastError(), what); }
 
+int g_pre_path = MHC_PATH_AUTO;
+
 }  // namespace mhc
 
 using namespace mhc;
@@ -110,7 +112,15 @@ mhc_status mhc_pre(const void* X, mhc_dtype x_dt, const void* phi, mhc_dtype phi
     }
     PreArgs a{X, x_dt, phi, phi_dt, {alpha[0], alpha[1], alpha[2]}, b, T, n, C, t_iters, eps,
               x_in, H_pre, H_post, H_res};
-    return launch_pre_fma(a, static_cast<cudaStream_t>(stream));
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool tc_ok = pre_tc_supported(a);
+    if (g_pre_path == MHC_PATH_TENSOR && !tc_ok) {
+        set_error("%s: the tensor-core path was forced but does not support this call "
+                  "(needs bf16 X and phi, n in {2,3,4}, C %% 512 == 0)", fn);
+        return MHC_ERR_UNSUPPORTED;
+    }
+    if (tc_ok && g_pre_path != MHC_PATH_FMA) return launch_pre_tc(a, s);
+    return launch_pre_fma(a, s);
 }
 
 mhc_status mhc_post(const void* X, const void* F_out, mhc_dtype dt, const float* H_post,
@@ -137,6 +147,22 @@ mhc_status mhc_post(const void* X, const void* F_out, mhc_dtype dt, const float*
                 !overlap(rXn, range_of(H_res, size_t(T) * n * n * 4)),
             MHC_ERR_INVALID_ARG, "%s: X_next overlaps F_out or a coefficient array", fn);
     return launch_post(X, F_out, dt, H_post, H_res, T, n, C, X_next, static_cast<cudaStream_t>(stream));
+}
+
+mhc_status mhc_set_path(mhc_path path)
+{
+    g_msg[0] = 0;
+    REQUIRE(path == MHC_PATH_AUTO || path == MHC_PATH_FMA || path == MHC_PATH_TENSOR,
+            MHC_ERR_INVALID_ARG, "mhc_set_path: unknown path %d", int(path));
+    g_pre_path = path;
+    return MHC_OK;
+}
+
+mhc_status mhc_set_wait_limit(long long polls)
+{
+    g_msg[0] = 0;
+    REQUIRE(polls >= 1, MHC_ERR_INVALID_ARG, "mhc_set_wait_limit: polls must be >= 1");
+    return cuda_status(cudaMemcpyToSymbol(g_wait_limit, &polls, sizeof(polls)), "mhc_set_wait_limit");
 }
 
 mhc_status mhc_sync_status(void* stream)

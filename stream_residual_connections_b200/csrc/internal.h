@@ -23,4 +23,12 @@ struct PreArgs {
 // CUDA-core (FMA) projection path: every n, dtype pair and C % 8 == 0.
 mhc_status launch_pre_fma(const PreArgs& a, cudaStream_t s);
 
+// Tensor-core path (TMA + tcgen05 + 8-CTA cluster): bf16 X and phi, n in
+// {2, 3, 4}, C % 512 == 0 and phi's per-CTA slice resident in shared memory.
+bool pre_tc_supported(const PreArgs& a);
+mhc_status launch_pre_tc(const PreArgs& a, cudaStream_t s);
+
+// Which mhc_pre path to take (MHC_PRE_PATH_*), process-wide.
+extern int g_pre_path;
+
 }  // namespace mhc

@@ -3,3 +3,4 @@
 #include "api.cu"
 #include "mhc_post.cu"
 #include "mhc_pre_fma.cu"
+#include "mhc_pre_tc.cu"
