@@ -236,7 +236,8 @@ def run_ours(args, world, rank, local):
             if a.dtype == np.uint16 else torch.from_numpy(a)
         return t.to(device)
 
-    X, F, phi = to_dev(inp["X"]), to_dev(inp["F"]), to_dev(inp["phi"])
+    X, F = to_dev(inp["X"]), to_dev(inp["F"])
+    phi = to_dev(np.ascontiguousarray(inp["phi"].T))        # the library's layout: phi^T [P][nC]
     b = torch.from_numpy(inp["b"]).to(device)
     alpha = inp["alpha"]
     x_in = torch.empty((T, C), dtype=torch.bfloat16, device=device)

@@ -69,7 +69,10 @@ int mhc_version(void);
  *   x_in[c] = sum_i H_pre[i] * X_t[i][c]
  *
  *   X      [T][n][C], dtype x_dt                       (read)
- *   phi    [n*C][P],  dtype phi_dt; columns pre n | post n | res n*n (read)
+ *   phi    [P][n*C],  dtype phi_dt: the projection matrix of Eq.(7) stored
+ *          transposed (the layout of a linear layer's weight): row p holds
+ *          the weights of logit p over vec(X_t); rows are pre n | post n |
+ *          res n*n, res row-major (read)
  *   alpha  HOST float[3] = (alpha_pre, alpha_post, alpha_res)
  *   b      [P] fp32                                    (read)
  *   x_in   [T][C], dtype x_dt                          (written)

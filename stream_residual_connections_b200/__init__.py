@@ -101,7 +101,8 @@ def _host3(alpha, count=3):
 
 def mhc_pre(X, phi, alpha, b, t_iters: int = 20, eps: float = 1e-6, *, x_in=None, H_pre=None,
             H_post=None, H_res=None, want_H_pre: bool = True, stream=None):
-    """Pre half of one mHC sublayer (see include/mhc.h).  X [T][n][C], phi [nC][n^2+2n],
+    """Pre half of one mHC sublayer (see include/mhc.h).  X [T][n][C], phi [n^2+2n][nC]
+    (the projection stored transposed, like a linear layer's weight),
     alpha: 3 host floats, b [n^2+2n] fp32.  Returns (x_in, H_pre, H_post, H_res)."""
     T, n, C = X.shape
     dev = X.device

@@ -7,8 +7,8 @@
 // (Eq.19); the F_pre contraction x_in = H_pre X closes the kernel.
 //
 // Each lane walks its share of the n*C row 8 (bf16) or 4 (fp32) elements at a
-// time, reading the matching rows of phi with 16-byte loads and keeping P fp32
-// accumulators.  A butterfly reduction gives every lane the full logits, so
+// time, reading the matching columns of every row of phi^T ([P][nC]) with
+// 16-byte loads and keeping P fp32 accumulators.  A butterfly reduction gives every lane the full logits, so
 // the small coefficient math runs redundantly per lane with no further
 // communication.  The row is then re-read (now mostly from L2) for x_in.
 //
@@ -24,7 +24,7 @@ template <typename TP> struct PhiVec { static constexpr int W = 16 / sizeof(TP);
 
 template <int N, typename TX, typename TP>
 __global__ void __launch_bounds__(256)
-pre_fma_kernel(const TX* __restrict__ X, const TP* __restrict__ phi, float a0, float a1, float a2,
+pre_fma_kernel(const TX* __restrict__ X, const TP* __restrict__ phiT, float a0, float a1, float a2,
                const float* __restrict__ b, int64_t T, int C, int t_iters, float eps,
                TX* __restrict__ x_in, float* __restrict__ Hpre, float* __restrict__ Hpost,
                float* __restrict__ Hres)
@@ -32,7 +32,7 @@ pre_fma_kernel(const TX* __restrict__ X, const TP* __restrict__ phi, float a0, f
     constexpr int P = N * N + 2 * N;
     constexpr int W = Vec<TX>::W;            // X elements per 16-byte load
     constexpr int PW = PhiVec<TP>::W;        // phi elements per 16-byte load
-    static_assert((W * P) % PW == 0, "phi rows of a vector step must fill 16-byte loads");
+    static_assert(W % PW == 0, "a vector step of X must cover whole 16-byte loads of phi");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t = int64_t(blockIdx.x) * (blockDim.x >> 5) + warp;
     if (t >= T) return;                       // whole warp leaves together
@@ -48,15 +48,14 @@ pre_fma_kernel(const TX* __restrict__ X, const TP* __restrict__ phi, float a0, f
         load16<false>(x + k0, xv);
 #pragma unroll
         for (int e = 0; e < W; ++e) ss = fmaf(xv[e], xv[e], ss);
-        const TP* prow = phi + k0 * P;       // W consecutive phi rows, W*P elements
 #pragma unroll
-        for (int q = 0; q < W * P; q += PW) {
-            float pv[PW];
-            load16<false>(prow + q, pv);
+        for (int p = 0; p < P; ++p) {        // row p of phi^T: the weights of logit p
 #pragma unroll
-            for (int e2 = 0; e2 < PW; ++e2) {
-                const int idx = q + e2;       // compile-time after unrolling
-                acc[idx % P] = fmaf(xv[idx / P], pv[e2], acc[idx % P]);
+            for (int h = 0; h < W; h += PW) {
+                float pv[PW];
+                load16<false>(phiT + int64_t(p) * K + k0 + h, pv);
+#pragma unroll
+                for (int e = 0; e < PW; ++e) acc[p] = fmaf(xv[h + e], pv[e], acc[p]);
             }
         }
     }

@@ -4,26 +4,30 @@
 // [mHC] section 4.3.1, Eq.(14)-(19), and F_pre := H_pre x_l.  Per token tile
 // of Mt <= 128 tokens, the 8 CTAs of a cluster split the C channels: CTA r
 // owns channels [r*C/8, (r+1)*C/8) of every stream, i.e. a K-slice of
-// n*C/8 elements of each token's n*C row.
+// n*C/8 elements of each token's n*C row, and phi's matching K-slice stays
+// resident in its shared memory for the whole (persistent) kernel.
 //
-//   warp 0   TMA producer: streams X[tile, stream i, 64-channel block] boxes
-//            (Mt rows x 128 B, 128-byte swizzle) through a 4-stage ring.
-//   warp 1   MMA issuer: D[Mt x NB] += X_chunk[Mt x 64] * phiT_chunk[NB x 64]^T
-//            (tcgen05.mma kind::f16, M = 128, fp32 accumulator in TMEM,
-//            double-buffered across tiles).  phiT (this CTA's K-slice of phi,
-//            transposed to K-major) stays resident in shared memory.
-//   warps 2-5 epilogue: the sum of squares of each row straight from the
-//            ring stage (Eq.15), the partial logits from TMEM, an exchange of
-//            the 8 partial (logits, sum of squares) rows through DSMEM, the
-//            coefficients of 16 tokens per CTA (Eq.16-19, Sinkhorn in
-//            registers), a DSMEM broadcast of H_pre, and x_in = H_pre X for
-//            this CTA's channels (re-reading the tile's X slice, which the
-//            cluster's recent loads keep in L2).
+// Warp roles (16 warps):
+//   0      TMA producer: X[tile, stream i, 64-channel block] boxes (Mt rows x
+//          128 B, 128-byte swizzle, L2 evict-last) through a 4-stage ring.
+//   1      MMA issuer: D[Mt x NB] += X_chunk[Mt x 64] * phiT_chunk[NB x 64]^T
+//          (tcgen05.mma kind::f16, M = 128, fp32 accumulator in TMEM,
+//          double-buffered across tiles).
+//   2-3    sum of squares of every row of every ring stage (Eq.15), handed to
+//          the epilogue through a double-buffered shared array.
+//   4-7    epilogue: partial logits from TMEM; exchange of the 8 partial
+//          (logits, sum of squares) rows through DSMEM; coefficients of 16
+//          tokens per CTA (Eq.16-19, Sinkhorn in registers); H_pre broadcast
+//          to the cluster through DSMEM.
+//   8-15   x_in = H_pre X for this CTA's channels, re-reading the tile's X
+//          slice while it is still in L2 (evict-first on this last read).
+// The roles meet only through mbarriers, so the TMA ring keeps streaming
+// while a tile's coefficients and x_in are being produced.
 //
-// HBM: X is read once by TMA; x_in and the coefficients are written once.
-// phi is read once per CTA.  Every mbarrier wait is bounded (g_wait_limit);
-// on expiry the kernel records MHC_ERR_TIMEOUT in the device error word,
-// drains its own copies in flight, frees TMEM and returns.
+// HBM: X is read once; x_in and the coefficients are written once; phi is
+// read once per CTA.  Every mbarrier wait is bounded (g_wait_limit); on
+// expiry the kernel records the timeout in the device error word, drains its
+// own copies and MMAs in flight, frees TMEM and returns.
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
@@ -38,8 +42,10 @@ constexpr int MROWS = 128;       // MMA M: token rows of one tile buffer
 constexpr int KC = 64;           // K elements per chunk (one 128-byte row)
 constexpr int STAGE_BYTES = MROWS * 128;
 constexpr int STAGES = 4;
-constexpr int NTHREADS = 192;    // 6 warps
-constexpr int EPI_THREADS = 128; // warps 2..5
+constexpr int NTHREADS = 512;
+constexpr int SS_WARP0 = 2, SS_WARPS = 2;
+constexpr int EPI_WARP0 = 4, EPI_WARPS = 4, EPI_THREADS = 128;
+constexpr int XIN_WARP0 = 8, XIN_WARPS = 8, XIN_THREADS = 256;
 constexpr int TOK_PER_CTA = MROWS / CL;  // tokens whose coefficients a CTA computes
 
 template <int N> struct Cfg {
@@ -50,8 +56,12 @@ template <int N> struct Cfg {
     static constexpr int TMEM_COLS = (2 * NB <= 32) ? 32 : (2 * NB <= 64 ? 64 : (2 * NB <= 128 ? 128 : 256));
 };
 
+enum Bar { B_FULL = 0, B_EMPTY = B_FULL + STAGES, B_TFULL = B_EMPTY + STAGES, B_TEMPTY = B_TFULL + 2,
+           B_SSFULL = B_TEMPTY + 2, B_SSEMPTY = B_SSFULL + 2, B_PART = B_SSEMPTY + 2, B_HPRE,
+           B_EPI, B_XIN, B_PHI, B_DRAIN, B_COUNT };
+
 struct Layout {
-    uint32_t phi, ring, part, hpre, bars, slot, total;
+    uint32_t phi, ring, part, ss, hpre, bars, slot, total;
 };
 
 template <int N>
@@ -61,17 +71,18 @@ __host__ __device__ inline Layout layout_for(int NQ) {
     L.phi = 0;
     L.ring = uint32_t(NQ) * G::R * 128;                      // multiple of 1024
     L.part = L.ring + STAGES * STAGE_BYTES;
-    L.hpre = L.part + MROWS * G::PS * 4;
-    L.bars = (L.hpre + MROWS * N * 4 + 15) / 16 * 16;
-    L.slot = L.bars + (2 * STAGES + 8) * 8;
+    L.ss = L.part + MROWS * G::PS * 4;
+    L.hpre = L.ss + 2 * MROWS * 4;
+    L.bars = (L.hpre + 2 * MROWS * N * 4 + 15) / 16 * 16;
+    L.slot = L.bars + B_COUNT * 8;
     L.total = L.slot + 16;
     return L;
 }
 
 template <int N>
 __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NTHREADS, 1)
-pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const bf16_t* __restrict__ X,
-              const bf16_t* __restrict__ phi, float a0, float a1, float a2,
+pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmPhi,
+              const bf16_t* __restrict__ X, float a0, float a1, float a2,
               const float* __restrict__ b, int64_t T, int C, int Mt, int num_tiles, int t_iters,
               float eps, bf16_t* __restrict__ x_in, float* __restrict__ Hpre,
               float* __restrict__ Hpost, float* __restrict__ Hres)
@@ -89,16 +100,21 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const bf16_t* __restrict_
     uint8_t* sphi = smem + L.phi;
     uint8_t* sring = smem + L.ring;
     float* spart = reinterpret_cast<float*>(smem + L.part);
-    float* shpre = reinterpret_cast<float*>(smem + L.hpre);
+    float* sss = reinterpret_cast<float*>(smem + L.ss);       // [2][MROWS]
+    float* shpre = reinterpret_cast<float*>(smem + L.hpre);   // [2][MROWS][N]
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
-    uint64_t* full = bars;
-    uint64_t* empty = bars + STAGES;
-    uint64_t* tfull = bars + 2 * STAGES;
-    uint64_t* tempty = tfull + 2;
-    uint64_t* part_ready = tempty + 2;
-    uint64_t* hpre_ready = part_ready + 1;
-    uint64_t* epi_sync = hpre_ready + 1;   // the 128 epilogue threads, twice per tile
-    uint64_t* drain = epi_sync + 1;        // MMA completion on the abort path
+    uint64_t* full = bars + B_FULL;
+    uint64_t* empty = bars + B_EMPTY;
+    uint64_t* tfull = bars + B_TFULL;
+    uint64_t* tempty = bars + B_TEMPTY;
+    uint64_t* ssfull = bars + B_SSFULL;
+    uint64_t* ssempty = bars + B_SSEMPTY;
+    uint64_t* part_ready = bars + B_PART;
+    uint64_t* hpre_ready = bars + B_HPRE;
+    uint64_t* epi_sync = bars + B_EPI;
+    uint64_t* xin_prog = bars + B_XIN;
+    uint64_t* phi_full = bars + B_PHI;
+    uint64_t* drain = bars + B_DRAIN;
     uint32_t* slot = reinterpret_cast<uint32_t*>(smem + L.slot);
     __shared__ int s_abort;
 
@@ -112,44 +128,41 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const bf16_t* __restrict_
         s_abort = 0;
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1 + EPI_THREADS / 32);
+            mbar_init(&empty[s], 1 + SS_WARPS);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], EPI_THREADS / 32);
+            mbar_init(&tempty[a], EPI_WARPS);
+            mbar_init(&ssfull[a], SS_WARPS);
+            mbar_init(&ssempty[a], EPI_WARPS);
         }
         mbar_init(part_ready, CL);
         mbar_init(hpre_ready, CL);
         mbar_init(epi_sync, EPI_THREADS);
+        mbar_init(xin_prog, XIN_WARPS);
+        mbar_init(phi_full, 1);
         mbar_init(drain, 1);
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(slot, G::TMEM_COLS);
-    if (warp == 0 && lane == 0) tma_prefetch(&tmX);
-
-    // Resident phiT: chunk q = (stream i, channel block cb) holds rows p < R of
-    // phi[i*C + c0 + cb*64 + kk][p] at kk, 128-byte rows, 16-byte groups XOR-swizzled by row.
-    for (int e = threadIdx.x; e < NQ * KC; e += NTHREADS) {
-        const int q = e / KC, kk = e % KC;
-        const int i = q / CB, cb = q % CB;
-        const int64_t k = int64_t(i) * C + c0 + cb * KC + kk;
-        uint8_t* rowbase = sphi + size_t(q) * R * 128;
-        const int grp = kk >> 3, within = (kk & 7) * 2;
-#pragma unroll 4
-        for (int p = 0; p < R; ++p) {
-            const bf16_t v = p < P ? phi[k * P + p] : bf16_t(0);
-            *reinterpret_cast<bf16_t*>(rowbase + p * 128 + ((grp ^ (p & 7)) << 4) + within) = v;
-        }
-    }
-    fence_proxy_async_smem();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *slot;
+    if (threadIdx.x == 0) {
+        tma_prefetch(&tmX);
+        tma_prefetch(&tmPhi);
+        // Resident phiT: chunk q = (stream i, channel block cb) holds rows p < R of
+        // phiT[p][i*C + c0 + cb*64 + 0..63] (rows >= P are zero-filled by the TMA).
+        mbar_arrive_expect_tx(phi_full, uint32_t(NQ) * R * 128);
+        for (int q = 0; q < NQ; ++q)
+            tma_load_2d(sphi + size_t(q) * R * 128, &tmPhi, phi_full, (q / CB) * C + c0 + (q % CB) * KC, 0);
+    }
     cluster_sync();   // every CTA's barriers are initialised before any remote arrive
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
+            const uint64_t keep = policy_evict_last();
             int s = 0;
             uint32_t ph = 0;
             int inflight_s[STAGES], inflight_ph[STAGES], n_issued = 0;
@@ -159,7 +172,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const bf16_t* __restrict_
                 for (int q = 0; q < NQ; ++q) {
                     if (!mbar_wait(&empty[s], ph ^ 1) || *(volatile int*)&s_abort) { ok = false; break; }
                     mbar_arrive_expect_tx(&full[s], uint32_t(Mt) * 128);
-                    tma_load_3d(sring + s * STAGE_BYTES, &tmX, &full[s], c0 + (q % CB) * KC, q / CB, t0);
+                    tma_load_3d_hint(sring + s * STAGE_BYTES, &tmX, &full[s], c0 + (q % CB) * KC, q / CB, t0, keep);
                     inflight_s[n_issued % STAGES] = s;
                     inflight_ph[n_issued % STAGES] = int(ph);
                     ++n_issued;
@@ -174,6 +187,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const bf16_t* __restrict_
                     mbar_wait(&full[inflight_s[j]], uint32_t(inflight_ph[j]), 1ll << 22);
             }
         }
+        if (lane == 1) mbar_wait(phi_full, 0, 1ll << 24);     // phiT copy settles before any exit
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -181,7 +195,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const bf16_t* __restrict_
             const uint32_t ring_a = smem_u32(sring), phi_a = smem_u32(sphi);
             int s = 0, it = 0;
             uint32_t ph = 0;
-            bool ok = true;
+            bool ok = mbar_wait(phi_full, 0);
             for (int tile = cluster_id; tile < num_tiles && ok; tile += nclusters, ++it) {
                 const int acc = it & 1;
                 if (!mbar_wait(&tempty[acc], (uint32_t((it >> 1) & 1)) ^ 1)) { ok = false; break; }
@@ -207,40 +221,53 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const bf16_t* __restrict_
                 mbar_wait(drain, 0, 1ll << 22);
             }
         }
-    } else {
-        // ------------------------------------------------------------ epilogue
-        const int et = threadIdx.x - 64;          // 0..127
-        const int qd = warp & 3;                  // TMEM lane quarter of this warp
-        const int m = qd * 32 + lane;             // token row within the tile
-        const float inv_K = 1.0f / float(N * C);
+    } else if (warp < EPI_WARP0) {
+        // ------------------------------------------------------------ sum of squares
+        const int r0 = (warp - SS_WARP0) * 32 + lane;   // rows r0 and r0 + 64
         int s = 0, it = 0;
         uint32_t ph = 0;
         for (int tile = cluster_id; tile < num_tiles; tile += nclusters, ++it) {
-            const int64_t t0 = int64_t(tile) * Mt;
-            bool ok = true;
-            // Eq.(15): sum of squares of this row's K-slice, from the ring stages
-            float ss = 0.0f;
-            for (int q = 0; q < NQ; ++q) {
+            const int acc = it & 1;
+            bool ok = mbar_wait(&ssempty[acc], (uint32_t((it >> 1) & 1)) ^ 1);
+            float ssa = 0.0f, ssb = 0.0f;
+            for (int q = 0; q < NQ && ok; ++q) {
                 if (!mbar_wait(&full[s], ph) || *(volatile int*)&s_abort) { ok = false; break; }
-                const uint4* row = reinterpret_cast<const uint4*>(sring + s * STAGE_BYTES + m * 128);
+                const uint4* ra = reinterpret_cast<const uint4*>(sring + s * STAGE_BYTES + r0 * 128);
+                const uint4* rb = reinterpret_cast<const uint4*>(sring + s * STAGE_BYTES + (r0 + 64) * 128);
 #pragma unroll
                 for (int g = 0; g < 8; ++g) {
-                    const uint4 v = row[g];
-                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                    const uint4 va = ra[g], vb = rb[g];
+                    const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {
-                        const float lo = bf16_lo(w[h]), hi = bf16_hi(w[h]);
-                        ss = fmaf(lo, lo, ss);
-                        ss = fmaf(hi, hi, ss);
+                        float x0 = bf16_lo(wa[h]), x1 = bf16_hi(wa[h]);
+                        ssa = fmaf(x0, x0, ssa); ssa = fmaf(x1, x1, ssa);
+                        x0 = bf16_lo(wb[h]); x1 = bf16_hi(wb[h]);
+                        ssb = fmaf(x0, x0, ssb); ssb = fmaf(x1, x1, ssb);
                     }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[s]);
                 if (++s == STAGES) { s = 0; ph ^= 1; }
             }
-            const int acc = it & 1;
-            if (ok && !mbar_wait(&tfull[acc], uint32_t((it >> 1) & 1))) ok = false;
             if (!ok) { s_abort = 1; break; }
+            sss[acc * MROWS + r0] = ssa;
+            sss[acc * MROWS + r0 + 64] = ssb;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ssfull[acc]);
+        }
+    } else if (warp < XIN_WARP0) {
+        // ------------------------------------------------------------ epilogue
+        const int et = threadIdx.x - EPI_WARP0 * 32;    // 0..127
+        const int qd = warp & 3;                        // TMEM lane quarter of this warp
+        const int m = qd * 32 + lane;                   // token row within the tile
+        const float inv_K = 1.0f / float(N * C);
+        int it = 0;
+        for (int tile = cluster_id; tile < num_tiles; tile += nclusters, ++it) {
+            const int64_t t0 = int64_t(tile) * Mt;
+            const int acc = it & 1;
+            const uint32_t par = uint32_t((it >> 1) & 1);
+            if (!mbar_wait(&tfull[acc], par) || !mbar_wait(&ssfull[acc], par)) { s_abort = 1; break; }
             tc_fence_after();
             float d[NB];
             const uint32_t taddr = tmem_base + (uint32_t(qd * 32) << 16) + uint32_t(acc * NB);
@@ -252,9 +279,10 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const bf16_t* __restrict_
 #pragma unroll
                 for (int j = 0; j < 16; ++j) d[c + j] = tmp[j];
             }
+            const float ss = sss[acc * MROWS + m];
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[acc]);
+            if (lane == 0) { mbar_arrive(&tempty[acc]); mbar_arrive(&ssempty[acc]); }
 
             // share this CTA's partial logits and sum of squares with the cluster
 #pragma unroll
@@ -263,7 +291,10 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const bf16_t* __restrict_
             asm volatile("fence.acq_rel.cluster;" ::: "memory");
             mbar_arrive(epi_sync);
             if (et == 0) {
-                if (!mbar_wait(epi_sync, 0)) { s_abort = 1; break; }
+                bool ok = mbar_wait(epi_sync, 0);
+                // the x_in warps have moved past tile it-1, so its H_pre buffer may be rewritten
+                if (ok && it >= 1) ok = mbar_wait(xin_prog, uint32_t((it - 1) & 1));
+                if (!ok) { s_abort = 1; break; }
                 for (uint32_t r = 0; r < CL; ++r) mbar_arrive_cluster(mapa(smem_u32(part_ready), r));
             }
             if (!mbar_wait<true>(part_ready, uint32_t(it & 1))) { s_abort = 1; break; }
@@ -303,8 +334,9 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const bf16_t* __restrict_
                     for (int i = 0; i < N; ++i)
 #pragma unroll
                         for (int k = 0; k < N; ++k) Hres[(t * N + i) * N + k] = m2[i][k];
+                    const uint32_t hoff = smem_u32(shpre + (acc * MROWS + j) * N);
                     for (uint32_t rr = 0; rr < CL; ++rr) {
-                        const uint32_t hb = mapa(smem_u32(shpre + j * N), rr);
+                        const uint32_t hb = mapa(hoff, rr);
 #pragma unroll
                         for (int i = 0; i < N; ++i) st_cluster_f32(hb + i * 4, hp[i]);
                     }
@@ -316,29 +348,50 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const bf16_t* __restrict_
                 if (!mbar_wait(epi_sync, 1)) { s_abort = 1; break; }
                 for (uint32_t r = 0; r < CL; ++r) mbar_arrive_cluster(mapa(smem_u32(hpre_ready), r));
             }
+            // the partial rows of this tile are no longer read once every CTA has its H_pre
             if (!mbar_wait<true>(hpre_ready, uint32_t(it & 1))) { s_abort = 1; break; }
-
-            // F_pre: x_in[t][c] = sum_i H_pre[t][i] X[t][i][c] for this CTA's channels
-            const int VPT = Cs / 8;                  // 16-byte vectors per token
+        }
+    } else {
+        // ------------------------------------------------------------ x_in
+        const int xt = threadIdx.x - XIN_WARP0 * 32;    // 0..255
+        const uint64_t drop = policy_evict_first();
+        const int VPT = Cs / 8;                          // 16-byte vectors per token
+        int it = 0;
+        for (int tile = cluster_id; tile < num_tiles; tile += nclusters, ++it) {
+            if (!mbar_wait<true>(hpre_ready, uint32_t(it & 1))) { s_abort = 1; break; }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(xin_prog);
+            const int64_t t0 = int64_t(tile) * Mt;
+            const float* hb = shpre + (it & 1) * MROWS * N;
             const int rows = int((T - t0) < int64_t(Mt) ? (T - t0) : int64_t(Mt));
             const int items = rows * VPT;
-#pragma unroll 2
-            for (int w = et; w < items; w += EPI_THREADS) {
-                const int tok = w / VPT, v = w - tok * VPT;
-                const int64_t t = t0 + tok;
-                const int c = c0 + v * 8;
-                float o[8];
+            for (int w0 = xt; w0 < items; w0 += 2 * XIN_THREADS) {
+                float xv[2][N][8];
+                int tok[2], cc[2];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) o[e] = 0.0f;
+                for (int u = 0; u < 2; ++u) {
+                    const int w = w0 + u * XIN_THREADS;
+                    const int wc = w < items ? w : items - 1;   // clamp; the store is skipped
+                    tok[u] = wc / VPT;
+                    cc[u] = c0 + (wc - tok[u] * VPT) * 8;
 #pragma unroll
-                for (int i = 0; i < N; ++i) {
-                    float xv[8];
-                    load16<false>(X + (t * N + i) * C + c, xv);
-                    const float h = shpre[tok * N + i];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) o[e] = fmaf(h, xv[e], o[e]);
+                    for (int i = 0; i < N; ++i)
+                        ldg16_hint(X + ((t0 + tok[u]) * N + i) * C + cc[u], xv[u][i], drop);
                 }
-                store16<false>(x_in + t * C + c, o);
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    if (w0 + u * XIN_THREADS >= items) break;
+                    float o[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) o[e] = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < N; ++i) {
+                        const float h = hb[tok[u] * N + i];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) o[e] = fmaf(h, xv[u][i][e], o[e]);
+                    }
+                    store16<false>(x_in + (t0 + tok[u]) * C + cc[u], o);
+                }
             }
         }
     }
@@ -418,22 +471,39 @@ static mhc_status launch_n(const PreArgs& a, cudaStream_t s)
         set_error("mhc_pre (tc): cuTensorMapEncodeTiled unavailable");
         return MHC_ERR_CUDA;
     }
-    CUtensorMap map;
-    const cuuint64_t dims[3] = {cuuint64_t(a.C), cuuint64_t(a.n), cuuint64_t(a.T)};
-    const cuuint64_t strides[2] = {cuuint64_t(a.C) * 2, cuuint64_t(a.n) * a.C * 2};
-    const cuuint32_t box[3] = {KC, 1, cuuint32_t(Mt)};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.X), dims, strides,
-                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) {
-        set_error("mhc_pre (tc): cuTensorMapEncodeTiled failed (%d)", int(r));
-        return MHC_ERR_CUDA;
+    using G = Cfg<N>;
+    CUtensorMap mapX, mapPhi;
+    {
+        const cuuint64_t dims[3] = {cuuint64_t(a.C), cuuint64_t(a.n), cuuint64_t(a.T)};
+        const cuuint64_t strides[2] = {cuuint64_t(a.C) * 2, cuuint64_t(a.n) * a.C * 2};
+        const cuuint32_t box[3] = {KC, 1, cuuint32_t(Mt)};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        CUresult r = enc(&mapX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.X), dims, strides,
+                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            set_error("mhc_pre (tc): cuTensorMapEncodeTiled(X) failed (%d)", int(r));
+            return MHC_ERR_CUDA;
+        }
+    }
+    {
+        const cuuint64_t K = cuuint64_t(a.n) * a.C;
+        const cuuint64_t dims[2] = {K, cuuint64_t(G::P)};
+        const cuuint64_t strides[1] = {K * 2};
+        const cuuint32_t box[2] = {KC, cuuint32_t(G::R)};
+        const cuuint32_t estr[2] = {1, 1};
+        CUresult r = enc(&mapPhi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.phi), dims, strides,
+                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            set_error("mhc_pre (tc): cuTensorMapEncodeTiled(phi) failed (%d)", int(r));
+            return MHC_ERR_CUDA;
+        }
     }
     kern<<<dim3(unsigned(nclusters * CL)), NTHREADS, size_t(smem), s>>>(
-        map, static_cast<const bf16_t*>(a.X), static_cast<const bf16_t*>(a.phi), a.alpha[0], a.alpha[1],
-        a.alpha[2], a.b, a.T, a.C, Mt, int(tiles64), a.t_iters, a.eps, static_cast<bf16_t*>(a.x_in),
-        a.H_pre, a.H_post, a.H_res);
+        mapX, mapPhi, static_cast<const bf16_t*>(a.X), a.alpha[0], a.alpha[1], a.alpha[2], a.b, a.T,
+        a.C, Mt, int(tiles64), a.t_iters, a.eps, static_cast<bf16_t*>(a.x_in), a.H_pre, a.H_post,
+        a.H_res);
     return launch_status("mhc_pre (tc) kernel");
 }
 

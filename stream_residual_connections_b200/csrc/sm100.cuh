@@ -99,6 +99,46 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
            "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
+// 2-D tile load into this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];"
+        :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+           "r"(c0), "r"(c1)
+        : "memory");
+}
+// L2 cache policies: keep (evict_last) data that is read again soon; drop
+// (evict_first) data on its last read.
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// 3-D tile load with an L2 cache policy.
+__device__ __forceinline__ void tma_load_3d_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int c0, int c1, int c2, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;"
+        :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+           "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+        : "memory");
+}
+// 16-byte global load (bf16 x 8 widened to fp32) with an L2 cache policy, no L1 allocation.
+__device__ __forceinline__ void ldg16_hint(const bf16_t* p, float (&v)[8], uint64_t policy) {
+    uint32_t a, b2, c, d;
+    asm volatile("ld.global.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(a), "=r"(b2), "=r"(c), "=r"(d) : "l"(p), "l"(policy));
+    v[0] = bf16_lo(a); v[1] = bf16_hi(a); v[2] = bf16_lo(b2); v[3] = bf16_hi(b2);
+    v[4] = bf16_lo(c); v[5] = bf16_hi(c); v[6] = bf16_lo(d); v[7] = bf16_hi(d);
+}
 // Make generic-proxy shared-memory writes visible to the async proxy (TMA, tensor core).
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -35,6 +35,12 @@ def dev(a: np.ndarray, device="cuda") -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a)).to(device)
 
 
+def phi_dev(phi: np.ndarray, device="cuda") -> torch.Tensor:
+    """Projection [nC][P] (the pages' orientation, as the oracle takes it) ->
+    device tensor in the library's layout, phi^T [P][nC]."""
+    return dev(np.ascontiguousarray(phi.T), device)
+
+
 def host(t: torch.Tensor) -> np.ndarray:
     """device tensor -> float64 numpy (exact widening)."""
     t = t.detach().cpu()

@@ -12,15 +12,15 @@ import torch
 import oracle
 import stream_residual_connections_b200 as M
 import synth
-from tests.parity import check_coeffs, check_mix, check_rounding, dev, host
+from tests.parity import check_coeffs, check_mix, check_rounding, dev, host, phi_dev
 
 pytestmark = pytest.mark.gpu
 
 
 def _run(inp, phi_dtype=None):
-    X, F, phi = dev(inp["X"]), dev(inp["F"]), dev(inp["phi"])
+    X, F, phi = dev(inp["X"]), dev(inp["F"]), phi_dev(inp["phi"])
     if phi_dtype == "f32":
-        phi = torch.from_numpy(oracle.widen(inp["phi"]).astype(np.float32)).cuda()
+        phi = phi_dev(oracle.widen(inp["phi"]).astype(np.float32))
     b = torch.from_numpy(inp["b"]).cuda()
     x_in, Hp, Ho, Hr = M.mhc_pre(X, phi, inp["alpha"], b, inp["t_iters"], inp["eps"])
     Xn = M.mhc_post(X, F, Ho, Hr)
@@ -91,7 +91,7 @@ def test_post_in_place():
     inp = synth.mhc_inputs(50, 4, 256, "bf16", seed=11)
     X, F = dev(inp["X"]), dev(inp["F"])
     b = torch.from_numpy(inp["b"]).cuda()
-    _, _, Ho, Hr = M.mhc_pre(X, dev(inp["phi"]), inp["alpha"], b)
+    _, _, Ho, Hr = M.mhc_pre(X, phi_dev(inp["phi"]), inp["alpha"], b)
     ref = M.mhc_post(X, F, Ho, Hr)
     out = M.mhc_post(X, F, Ho, Hr, X_next=X)
     torch.cuda.synchronize()
@@ -101,7 +101,7 @@ def test_post_in_place():
 
 def test_empty_T_is_a_no_op():
     X = torch.zeros((0, 4, 64), dtype=torch.bfloat16, device="cuda")
-    phi = torch.zeros((256, 24), dtype=torch.bfloat16, device="cuda")
+    phi = torch.zeros((24, 256), dtype=torch.bfloat16, device="cuda")
     b = torch.zeros(24, device="cuda")
     x_in, *_ = M.mhc_pre(X, phi, [0.01] * 3, b)
     assert x_in.shape == (0, 64)
@@ -109,7 +109,7 @@ def test_empty_T_is_a_no_op():
                torch.zeros((0, 4), device="cuda"), torch.zeros((0, 4, 4), device="cuda"))
 
 
-def test_plain_residual_and_permutation_reduction_bit_exact():
+def test_plain_residual_and_permutation_reduction_exact():
     """mHC page Eq.(1) vs Eq.(3): alpha = 0 with +-40 biases gives H_res = P_sigma,
     H_pre = e_2, H_post = 1; x_in = X[2] and X_next[i] = X[sigma(i)] + F, both
     bit-exact after the single bf16 rounding."""
@@ -128,7 +128,11 @@ def test_plain_residual_and_permutation_reduction_bit_exact():
     X, F = oracle.widen(inp["X"]), oracle.widen(inp["F"])
     np.testing.assert_array_equal(got["x_in"], X[:, 2])
     expect = oracle.widen(synth.f32_to_bf16_bits((X[:, sig] + F[:, None, :]).astype(np.float32)))
-    np.testing.assert_array_equal(got["X_next"], expect)
+    # bit-exact wherever X[sigma(i)] + F is not 0; where it cancels, the off-diagonal
+    # H_res weights exp(-80) (the oracle's too) leave a value of order 1e-35
+    nz = expect != 0
+    np.testing.assert_array_equal(got["X_next"][nz], expect[nz])
+    assert np.abs(got["X_next"][~nz]).max(initial=0.0) < 1e-30
     np.testing.assert_allclose(got["H_res"], np.broadcast_to(np.eye(n)[sig], (T, n, n)), atol=1e-30)
 
 
@@ -196,7 +200,7 @@ def test_bounded_wait_expiry_is_reported_and_context_survives(restore_path):
     the next normal call is correct."""
     M.mhc_set_path(M.MHC_PATH_TENSOR)
     inp = synth.mhc_inputs(2000, 4, 2048, "bf16", seed=23)
-    X, phi = dev(inp["X"]), dev(inp["phi"])
+    X, phi = dev(inp["X"]), phi_dev(inp["phi"])
     b = torch.from_numpy(inp["b"]).cuda()
     M.mhc_sync_status()
     M.mhc_set_wait_limit(1)
