@@ -106,6 +106,45 @@ __device__ __forceinline__ void sinkhorn_regs(float (&m)[N][N], int iters) {
     }
 }
 
+// Row-parallel Sinkhorn-Knopp over an aligned group of 8 lanes (N <= 8):
+// lane g < N of the group holds row g of the logits in `row`; lanes g >= N
+// hold anything and end with zeros.  Same arithmetic as sinkhorn_regs (per
+// column maximum shift when iters >= 1, then `iters` x {columns, rows}); the
+// column sums are butterfly reductions over the 8 lanes.  Every lane of the
+// warp must call it (it shuffles over the full warp).
+template <int N>
+__device__ __forceinline__ void sinkhorn_group8(float (&row)[N], int g, int iters) {
+    const bool live = g < N;
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+        float mx = live ? row[j] : -INFINITY;
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+        if (iters == 0) mx = 0.0f;
+        row[j] = live ? expf(row[j] - mx) : 0.0f;
+    }
+    for (int it = 0; it < iters; ++it) {
+        float cs[N];
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+            cs[j] = row[j];
+            cs[j] += __shfl_xor_sync(0xffffffffu, cs[j], 1);
+            cs[j] += __shfl_xor_sync(0xffffffffu, cs[j], 2);
+            cs[j] += __shfl_xor_sync(0xffffffffu, cs[j], 4);
+        }
+        float rs = 0.0f;
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+            row[j] *= 1.0f / cs[j];
+            rs += row[j];
+        }
+        const float inv = live ? 1.0f / rs : 0.0f;
+#pragma unroll
+        for (int j = 0; j < N; ++j) row[j] *= inv;
+    }
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -2,32 +2,34 @@
 // of 8 CTAs sharing partial sums through distributed shared memory).
 //
 // [mHC] section 4.3.1, Eq.(14)-(19), and F_pre := H_pre x_l.  Per token tile
-// of Mt <= 128 tokens, the 8 CTAs of a cluster split the C channels: CTA r
+// of Mt <= 64 tokens, the 8 CTAs of a cluster split the C channels: CTA r
 // owns channels [r*C/8, (r+1)*C/8) of every stream, i.e. a K-slice of
 // n*C/8 elements of each token's n*C row, and phi's matching K-slice stays
 // resident in its shared memory for the whole (persistent) kernel.
 //
 // Warp roles (16 warps):
 //   0      TMA producer: X[tile, stream i, 64-channel block] boxes (Mt rows x
-//          128 B, 128-byte swizzle, L2 evict-last) through a 4-stage ring.
-//   1      MMA issuer: D[Mt x NB] += X_chunk[Mt x 64] * phiT_chunk[NB x 64]^T
-//          (tcgen05.mma kind::f16, M = 128, fp32 accumulator in TMEM,
-//          double-buffered across tiles).
-//   2-3    sum of squares of every row of every ring stage (Eq.15), handed to
-//          the epilogue through a double-buffered shared array.
-//   4-7    epilogue: partial logits from TMEM; exchange of the 8 partial
-//          (logits, sum of squares) rows through DSMEM; coefficients of 16
-//          tokens per CTA (Eq.16-19, Sinkhorn in registers); H_pre broadcast
-//          to the cluster through DSMEM.
-//   8-15   x_in = H_pre X for this CTA's channels, re-reading the tile's X
-//          slice while it is still in L2 (evict-first on this last read).
-// The roles meet only through mbarriers, so the TMA ring keeps streaming
-// while a tile's coefficients and x_in are being produced.
+//          128 B, 128-byte swizzle, L2 evict-last) through an 8-stage ring;
+//          it runs at most LAG tiles ahead of the x_in warps, which keeps the
+//          x_in re-read inside L2.
+//   1      MMA issuer: D[128 x NB] += X_chunk[128 x 64] * phiT_chunk[NB x 64]^T
+//          (tcgen05.mma kind::f16, fp32 accumulator in TMEM, double-buffered
+//          across tiles; rows >= Mt are never read).
+//   2-3    sum of squares of every tile row of every ring stage (Eq.15),
+//          handed to the epilogue through a double-buffered shared array.
+//   4-5    epilogue: partial logits from TMEM; exchange of the 8 partial
+//          (logits, sum of squares) rows through DSMEM; coefficients of 8
+//          tokens per CTA (Eq.16-19; a row-parallel Sinkhorn over 8 lanes);
+//          H_pre broadcast to the cluster through DSMEM.
+//   6-15   x_in = H_pre X for this CTA's channels, re-reading the tile's X
+//          slice from L2 (evict-first on this last read).
+// The roles meet only through mbarriers and one progress counter, so the TMA
+// ring keeps streaming while a tile's coefficients and x_in are produced.
 //
 // HBM: X is read once; x_in and the coefficients are written once; phi is
-// read once per CTA.  Every mbarrier wait is bounded (g_wait_limit); on
-// expiry the kernel records the timeout in the device error word, drains its
-// own copies and MMAs in flight, frees TMEM and returns.
+// read once per CTA.  Every wait is bounded (g_wait_limit); on expiry the
+// kernel records the timeout in the device error word, drains its own copies
+// and MMAs in flight, frees TMEM and returns.
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
@@ -38,21 +40,25 @@ namespace pretc {
 using namespace sm100;
 
 constexpr int CL = 8;            // CTAs per cluster (channel split)
-constexpr int MROWS = 128;       // MMA M: token rows of one tile buffer
+constexpr int MROWS = 128;       // MMA M (TMEM lanes); a tile uses the first Mt <= MT_CAP rows
+constexpr int MT_CAP = 64;       // token rows per tile: bounds the L2 footprint of the x_in re-read
 constexpr int KC = 64;           // K elements per chunk (one 128-byte row)
-constexpr int STAGE_BYTES = MROWS * 128;
-constexpr int STAGES = 4;
+constexpr int STAGE_BYTES = MT_CAP * 128;
+constexpr int STAGES = 8;
 constexpr int NTHREADS = 512;
-constexpr int SS_WARP0 = 2, SS_WARPS = 2;
-constexpr int EPI_WARP0 = 4, EPI_WARPS = 4, EPI_THREADS = 128;
-constexpr int XIN_WARP0 = 8, XIN_WARPS = 8, XIN_THREADS = 256;
-constexpr int TOK_PER_CTA = MROWS / CL;  // tokens whose coefficients a CTA computes
+constexpr int SS_WARP0 = 2, SS_WARPS = 2;                  // one tile row per thread
+constexpr int EPI_WARP0 = 4, EPI_WARPS = 2, EPI_THREADS = 64;
+constexpr int XIN_WARP0 = 6, XIN_WARPS = 10, XIN_THREADS = 320;
+constexpr int TOK_PER_CTA = MT_CAP / CL;  // tokens whose coefficients a CTA computes
+constexpr int XIN_UNROLL = 4;             // x_in vectors in flight per thread
+constexpr int LAG = 2;                    // tiles the TMA stream may run ahead of x_in
 
 template <int N> struct Cfg {
     static constexpr int P = N * N + 2 * N;
     static constexpr int R = (P + 7) / 8 * 8;      // phiT rows stored per chunk
     static constexpr int NB = (P + 15) / 16 * 16;  // MMA N
     static constexpr int PS = P + 1;               // partial row: P logits + sum of squares
+    static constexpr int PSP = (PS + 3) / 4 * 4;   // ... padded to 16-byte multiples
     static constexpr int TMEM_COLS = (2 * NB <= 32) ? 32 : (2 * NB <= 64 ? 64 : (2 * NB <= 128 ? 128 : 256));
 };
 
@@ -71,11 +77,16 @@ __host__ __device__ inline Layout layout_for(int NQ) {
     L.phi = 0;
     L.ring = uint32_t(NQ) * G::R * 128;                      // multiple of 1024
     L.part = L.ring + STAGES * STAGE_BYTES;
-    L.ss = L.part + MROWS * G::PS * 4;
-    L.hpre = L.ss + 2 * MROWS * 4;
-    L.bars = (L.hpre + 2 * MROWS * N * 4 + 15) / 16 * 16;
+    L.ss = L.part + MT_CAP * G::PSP * 4;
+    L.hpre = L.ss + 2 * MT_CAP * 4;
+    L.bars = (L.hpre + 2 * MT_CAP * N * 4 + 15) / 16 * 16;
     L.slot = L.bars + B_COUNT * 8;
     L.total = L.slot + 16;
+    // The MMA reads 128 rows from a stage's base: the last stage's rows past
+    // MT_CAP must still be inside this CTA's shared memory (their products land
+    // in accumulator rows that are never read).
+    const uint32_t mma_end = L.part + (MROWS - MT_CAP) * 128;
+    if (L.total < mma_end) L.total = mma_end;
     return L;
 }
 
@@ -88,7 +99,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
               float* __restrict__ Hpost, float* __restrict__ Hres)
 {
     using G = Cfg<N>;
-    constexpr int P = G::P, R = G::R, NB = G::NB, PS = G::PS;
+    constexpr int P = G::P, R = G::R, NB = G::NB, PS = G::PS, PSP = G::PSP;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte-swizzle atoms
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -100,8 +111,8 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     uint8_t* sphi = smem + L.phi;
     uint8_t* sring = smem + L.ring;
     float* spart = reinterpret_cast<float*>(smem + L.part);
-    float* sss = reinterpret_cast<float*>(smem + L.ss);       // [2][MROWS]
-    float* shpre = reinterpret_cast<float*>(smem + L.hpre);   // [2][MROWS][N]
+    float* sss = reinterpret_cast<float*>(smem + L.ss);       // [2][MT_CAP]
+    float* shpre = reinterpret_cast<float*>(smem + L.hpre);   // [2][MT_CAP][N]
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
     uint64_t* full = bars + B_FULL;
     uint64_t* empty = bars + B_EMPTY;
@@ -117,6 +128,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     uint64_t* drain = bars + B_DRAIN;
     uint32_t* slot = reinterpret_cast<uint32_t*>(smem + L.slot);
     __shared__ int s_abort;
+    __shared__ int s_xin_done;   // x_in warp-tiles finished (monotonic)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -126,6 +138,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
 
     if (threadIdx.x == 0) {
         s_abort = 0;
+        s_xin_done = 0;
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1 + SS_WARPS);
@@ -167,8 +180,19 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             uint32_t ph = 0;
             int inflight_s[STAGES], inflight_ph[STAGES], n_issued = 0;
             bool ok = true;
-            for (int tile = cluster_id; tile < num_tiles && ok; tile += nclusters) {
+            int it = 0;
+            for (int tile = cluster_id; tile < num_tiles && ok; tile += nclusters, ++it) {
                 const int t0 = tile * Mt;
+                // keep the re-read of tile it-LAG in L2: do not run further ahead of x_in
+                if (it >= LAG) {
+                    const int need = XIN_WARPS * (it - LAG + 1);
+                    long long k = 0;
+                    while (*(volatile int*)&s_xin_done < need && !*(volatile int*)&s_abort && k < g_wait_limit) {
+                        __nanosleep(64);
+                        ++k;
+                    }
+                    if (k >= g_wait_limit) { atomicOr(&g_device_error, 1u); ok = false; break; }
+                }
                 for (int q = 0; q < NQ; ++q) {
                     if (!mbar_wait(&empty[s], ph ^ 1) || *(volatile int*)&s_abort) { ok = false; break; }
                     mbar_arrive_expect_tx(&full[s], uint32_t(Mt) * 128);
@@ -223,7 +247,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         }
     } else if (warp < EPI_WARP0) {
         // ------------------------------------------------------------ sum of squares
-        const int r0 = (warp - SS_WARP0) * 32 + lane;   // rows r0 and r0 + 64
+        const int r0 = (warp - SS_WARP0) * 32 + lane;   // tile row of this thread
         int s = 0, it = 0;
         uint32_t ph = 0;
         for (int tile = cluster_id; tile < num_tiles; tile += nclusters, ++it) {
@@ -233,10 +257,9 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             for (int q = 0; q < NQ && ok; ++q) {
                 if (!mbar_wait(&full[s], ph) || *(volatile int*)&s_abort) { ok = false; break; }
                 const uint4* ra = reinterpret_cast<const uint4*>(sring + s * STAGE_BYTES + r0 * 128);
-                const uint4* rb = reinterpret_cast<const uint4*>(sring + s * STAGE_BYTES + (r0 + 64) * 128);
 #pragma unroll
-                for (int g = 0; g < 8; ++g) {
-                    const uint4 va = ra[g], vb = rb[g];
+                for (int g = 0; g < 8; g += 2) {
+                    const uint4 va = ra[g], vb = ra[g + 1];
                     const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {
@@ -251,15 +274,14 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 if (++s == STAGES) { s = 0; ph ^= 1; }
             }
             if (!ok) { s_abort = 1; break; }
-            sss[acc * MROWS + r0] = ssa;
-            sss[acc * MROWS + r0 + 64] = ssb;
+            sss[acc * MT_CAP + r0] = ssa + ssb;
             __syncwarp();
             if (lane == 0) mbar_arrive(&ssfull[acc]);
         }
     } else if (warp < XIN_WARP0) {
         // ------------------------------------------------------------ epilogue
-        const int et = threadIdx.x - EPI_WARP0 * 32;    // 0..127
-        const int qd = warp & 3;                        // TMEM lane quarter of this warp
+        const int et = threadIdx.x - EPI_WARP0 * 32;    // 0..63
+        const int qd = warp & 3;                        // TMEM lane quarter of this warp (0, 1)
         const int m = qd * 32 + lane;                   // token row within the tile
         const float inv_K = 1.0f / float(N * C);
         int it = 0;
@@ -279,15 +301,22 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
 #pragma unroll
                 for (int j = 0; j < 16; ++j) d[c + j] = tmp[j];
             }
-            const float ss = sss[acc * MROWS + m];
+            const float ss = sss[acc * MT_CAP + m];
             tc_fence_before();
             __syncwarp();
             if (lane == 0) { mbar_arrive(&tempty[acc]); mbar_arrive(&ssempty[acc]); }
 
             // share this CTA's partial logits and sum of squares with the cluster
+            float* prow = spart + m * PSP;
 #pragma unroll
-            for (int p = 0; p < P; ++p) spart[m * PS + p] = d[p];
-            spart[m * PS + P] = ss;
+            for (int p = 0; p < PSP; p += 4) {
+                float4 w4;
+                w4.x = p + 0 < P ? d[p + 0] : (p + 0 == P ? ss : 0.0f);
+                w4.y = p + 1 < P ? d[p + 1] : (p + 1 == P ? ss : 0.0f);
+                w4.z = p + 2 < P ? d[p + 2] : (p + 2 == P ? ss : 0.0f);
+                w4.w = p + 3 < P ? d[p + 3] : (p + 3 == P ? ss : 0.0f);
+                *reinterpret_cast<float4*>(prow + p) = w4;
+            }
             asm volatile("fence.acq_rel.cluster;" ::: "memory");
             mbar_arrive(epi_sync);
             if (et == 0) {
@@ -299,47 +328,49 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             }
             if (!mbar_wait<true>(part_ready, uint32_t(it & 1))) { s_abort = 1; break; }
 
-            // coefficients of 16 tokens: lane group of 8 = one token, one source CTA per lane
+            // Coefficients of TOK_PER_CTA tokens: a group of 8 lanes per token; lane g
+            // fetches the partial row of CTA g, the group reduces, then lane g < N
+            // carries row g of H_res through a row-parallel Sinkhorn.
             {
-                const int jj = et >> 3, src = et & 7;
+                const int jj = et >> 3, g = et & 7;
                 const int j = int(rank) * TOK_PER_CTA + jj;     // row within the tile
-                const uint32_t pbase = mapa(smem_u32(spart + j * PS), uint32_t(src));
-                float v[PS];
+                const uint32_t pbase = mapa(smem_u32(spart + j * PSP), uint32_t(g));
+                float v[PSP];
 #pragma unroll
-                for (int p = 0; p < PS; ++p) v[p] = ld_cluster_f32(pbase + p * 4);
+                for (int p = 0; p < PSP; p += 4) {
+                    const float4 f4 = ld_cluster_f32x4(pbase + p * 4);
+                    v[p] = f4.x; v[p + 1] = f4.y; v[p + 2] = f4.z; v[p + 3] = f4.w;
+                }
 #pragma unroll
                 for (int p = 0; p < PS; ++p) {
                     v[p] += __shfl_xor_sync(0xffffffffu, v[p], 1);
                     v[p] += __shfl_xor_sync(0xffffffffu, v[p], 2);
                     v[p] += __shfl_xor_sync(0xffffffffu, v[p], 4);
                 }
-                const int64_t t = t0 + j;
-                if (src == 0 && j < Mt && t < T) {
-                    const float r = sqrtf(v[P] * inv_K + eps);                     // Eq.(15)
-                    const float inv_r = 1.0f / r;
-                    float hp[N], m2[N][N];
+                const float r = sqrtf(v[P] * inv_K + eps);                     // Eq.(15)
+                const float inv_r = 1.0f / r;
+                float zpre = 0.0f, zpost = 0.0f, row[N];
 #pragma unroll
-                    for (int i = 0; i < N; ++i) {
-                        hp[i] = sigmoidf_(a0 * v[i] * inv_r + __ldg(b + i));                   // Eq.(17)
-                        Hpost[t * N + i] = 2.0f * sigmoidf_(a1 * v[N + i] * inv_r + __ldg(b + N + i)); // Eq.(18)
-                        if (Hpre) Hpre[t * N + i] = hp[i];
-                    }
+                for (int k = 0; k < N; ++k) row[k] = 0.0f;
 #pragma unroll
-                    for (int i = 0; i < N; ++i)
+                for (int i = 0; i < N; ++i)
+                    if (g == i) {
+                        zpre = a0 * v[i] * inv_r + __ldg(b + i);                   // Eq.(16)
+                        zpost = a1 * v[N + i] * inv_r + __ldg(b + N + i);
 #pragma unroll
                         for (int k = 0; k < N; ++k)
-                            m2[i][k] = a2 * v[2 * N + i * N + k] * inv_r + __ldg(b + 2 * N + i * N + k);
-                    sinkhorn_regs<N>(m2, t_iters);                                    // Eq.(19)
-#pragma unroll
-                    for (int i = 0; i < N; ++i)
-#pragma unroll
-                        for (int k = 0; k < N; ++k) Hres[(t * N + i) * N + k] = m2[i][k];
-                    const uint32_t hoff = smem_u32(shpre + (acc * MROWS + j) * N);
-                    for (uint32_t rr = 0; rr < CL; ++rr) {
-                        const uint32_t hb = mapa(hoff, rr);
-#pragma unroll
-                        for (int i = 0; i < N; ++i) st_cluster_f32(hb + i * 4, hp[i]);
+                            row[k] = a2 * v[2 * N + i * N + k] * inv_r + __ldg(b + 2 * N + i * N + k);
                     }
+                sinkhorn_group8<N>(row, g, t_iters);                               // Eq.(19)
+                const int64_t t = t0 + j;
+                if (g < N && j < Mt && t < T) {
+                    const float hp = sigmoidf_(zpre);                              // Eq.(17)
+                    Hpost[t * N + g] = 2.0f * sigmoidf_(zpost);                    // Eq.(18)
+                    if (Hpre) Hpre[t * N + g] = hp;
+#pragma unroll
+                    for (int k = 0; k < N; ++k) Hres[(t * N + g) * N + k] = row[k];
+                    const uint32_t hoff = smem_u32(shpre + (acc * MT_CAP + j) * N + g);
+                    for (uint32_t rr = 0; rr < CL; ++rr) st_cluster_f32(mapa(hoff, rr), hp);
                 }
             }
             asm volatile("fence.acq_rel.cluster;" ::: "memory");
@@ -353,7 +384,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         }
     } else {
         // ------------------------------------------------------------ x_in
-        const int xt = threadIdx.x - XIN_WARP0 * 32;    // 0..255
+        const int xt = threadIdx.x - XIN_WARP0 * 32;    // 0..XIN_THREADS-1
         const uint64_t drop = policy_evict_first();
         const int VPT = Cs / 8;                          // 16-byte vectors per token
         int it = 0;
@@ -362,24 +393,24 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             __syncwarp();
             if (lane == 0) mbar_arrive(xin_prog);
             const int64_t t0 = int64_t(tile) * Mt;
-            const float* hb = shpre + (it & 1) * MROWS * N;
+            const float* hb = shpre + (it & 1) * MT_CAP * N;
             const int rows = int((T - t0) < int64_t(Mt) ? (T - t0) : int64_t(Mt));
             const int items = rows * VPT;
-            for (int w0 = xt; w0 < items; w0 += 2 * XIN_THREADS) {
-                float xv[2][N][8];
-                int tok[2], cc[2];
+            for (int w0 = xt; w0 < items; w0 += XIN_UNROLL * XIN_THREADS) {
+                uint4 raw[XIN_UNROLL][N];
+                int tok[XIN_UNROLL], cc[XIN_UNROLL];
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
+                for (int u = 0; u < XIN_UNROLL; ++u) {
                     const int w = w0 + u * XIN_THREADS;
                     const int wc = w < items ? w : items - 1;   // clamp; the store is skipped
                     tok[u] = wc / VPT;
                     cc[u] = c0 + (wc - tok[u] * VPT) * 8;
 #pragma unroll
                     for (int i = 0; i < N; ++i)
-                        ldg16_hint(X + ((t0 + tok[u]) * N + i) * C + cc[u], xv[u][i], drop);
+                        raw[u][i] = ldg16_raw_hint(X + ((t0 + tok[u]) * N + i) * C + cc[u], drop);
                 }
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
+                for (int u = 0; u < XIN_UNROLL; ++u) {
                     if (w0 + u * XIN_THREADS >= items) break;
                     float o[8];
 #pragma unroll
@@ -387,12 +418,18 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
 #pragma unroll
                     for (int i = 0; i < N; ++i) {
                         const float h = hb[tok[u] * N + i];
+                        const uint32_t w4[4] = {raw[u][i].x, raw[u][i].y, raw[u][i].z, raw[u][i].w};
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) o[e] = fmaf(h, xv[u][i][e], o[e]);
+                        for (int e = 0; e < 4; ++e) {
+                            o[2 * e] = fmaf(h, bf16_lo(w4[e]), o[2 * e]);
+                            o[2 * e + 1] = fmaf(h, bf16_hi(w4[e]), o[2 * e + 1]);
+                        }
                     }
                     store16<false>(x_in + (t0 + tok[u]) * C + cc[u], o);
                 }
             }
+            __syncwarp();
+            if (lane == 0) atomicAdd(&s_xin_done, 1);
         }
     }
 
@@ -459,10 +496,10 @@ static mhc_status launch_n(const PreArgs& a, cudaStream_t s)
         max_clusters = nc;
     }
     // Token tiles of Mt <= 128 rows, sized so that every cluster gets the same number.
-    const int64_t rounds = (a.T + int64_t(max_clusters) * MROWS - 1) / (int64_t(max_clusters) * MROWS);
+    const int64_t rounds = (a.T + int64_t(max_clusters) * MT_CAP - 1) / (int64_t(max_clusters) * MT_CAP);
     const int64_t per_round = (a.T + rounds - 1) / rounds;                     // tokens per round
     int Mt = int((per_round + max_clusters - 1) / max_clusters);
-    if (Mt > MROWS) Mt = MROWS;
+    if (Mt > MT_CAP) Mt = MT_CAP;
     const int64_t tiles64 = (a.T + Mt - 1) / Mt;
     const int nclusters = int(tiles64 < max_clusters ? tiles64 : max_clusters);
 

@@ -38,6 +38,16 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
 __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(addr), "f"(v) : "memory");
 }
+__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_cluster_f32x4(uint32_t addr, float4 v) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};"
+                 :: "r"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
+}
 
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -138,6 +148,13 @@ __device__ __forceinline__ void ldg16_hint(const bf16_t* p, float (&v)[8], uint6
                  : "=r"(a), "=r"(b2), "=r"(c), "=r"(d) : "l"(p), "l"(policy));
     v[0] = bf16_lo(a); v[1] = bf16_hi(a); v[2] = bf16_lo(b2); v[3] = bf16_hi(b2);
     v[4] = bf16_lo(c); v[5] = bf16_hi(c); v[6] = bf16_lo(d); v[7] = bf16_hi(d);
+}
+// Raw 16-byte global load with an L2 cache policy, no L1 allocation.
+__device__ __forceinline__ uint4 ldg16_raw_hint(const void* p, uint64_t policy) {
+    uint4 v;
+    asm volatile("ld.global.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p), "l"(policy));
+    return v;
 }
 // Make generic-proxy shared-memory writes visible to the async proxy (TMA, tensor core).
 __device__ __forceinline__ void fence_proxy_async_smem() {
