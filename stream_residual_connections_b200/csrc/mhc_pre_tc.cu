@@ -52,6 +52,7 @@ constexpr int XIN_WARP0 = 6, XIN_WARPS = 10, XIN_THREADS = 320;
 constexpr int TOK_PER_CTA = MT_CAP / CL;  // tokens whose coefficients a CTA computes
 constexpr int XIN_UNROLL = 4;             // x_in vectors in flight per thread
 constexpr int LAG = 2;                    // tiles the TMA stream may run ahead of x_in
+static_assert(TOK_PER_CTA * 8 <= EPI_THREADS, "one 8-lane group per coefficient token");
 
 template <int N> struct Cfg {
     static constexpr int P = N * N + 2 * N;
@@ -363,7 +364,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     }
                 sinkhorn_group8<N>(row, g, t_iters);                               // Eq.(19)
                 const int64_t t = t0 + j;
-                if (g < N && j < Mt && t < T) {
+                if (g < N && jj < TOK_PER_CTA && j < Mt && t < T) {
                     const float hp = sigmoidf_(zpre);                              // Eq.(17)
                     Hpost[t * N + g] = 2.0f * sigmoidf_(zpost);                    // Eq.(18)
                     if (Hpre) Hpre[t * N + g] = hp;
