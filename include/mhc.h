@@ -102,6 +102,25 @@ mhc_status mhc_pre(const void* X, mhc_dtype x_dt, const void* phi, mhc_dtype phi
 mhc_status mhc_post(const void* X, const void* F_out, mhc_dtype dt, const float* H_post,
                     const float* H_res, int64_t T, int n, int C, void* X_next, void* stream);
 
+/*
+ * xhc_conv_gs -- temporal feature augmentation of the xHC write-back.
+ * [xHC] "temporal feature augmentation": r causal depthwise convolutions of
+ * the sublayer output and Gram-Schmidt orthogonalisation of the Kr = r + 1
+ * components per token:
+ *   a_0 = F_out[t]; a_j[c] = sum_{s<kappa_j} w_j[s][c] * F_out[t-s][c]
+ *        (terms with t-s before the start of t's sequence are zero; sequences
+ *        of seq_len tokens are laid end to end, seq_len = T for one sequence)
+ *   v_0 = a_0; v_j = a_j - sum_{i<j} <a_j, v_i>/<v_i, v_i> v_i  (a zero v_i adds nothing)
+ *
+ *   F_out  [T][C], dtype dt (read)
+ *   conv_w fp32, the r weight arrays w_j [kappa_j][C] concatenated (read)
+ *   kappa  HOST int[r], 1 <= kappa_j <= 64;  1 <= r <= 4
+ *   V      [T][Kr][C] fp32: V[t][j] = v_j (written; must not overlap an input)
+ * The inner products are per token over the C channels.
+ */
+mhc_status xhc_conv_gs(const void* F_out, mhc_dtype dt, const float* conv_w, const int* kappa,
+                       int r, int64_t T, int C, int64_t seq_len, float* V, void* stream);
+
 /* Kernel selection for the projection of mhc_pre. */
 typedef enum {
     MHC_PATH_AUTO = 0,    /* tensor cores where supported, else CUDA cores (default) */

@@ -46,8 +46,10 @@ def _load():
     L.mhc_post.argtypes = [vp, vp, i32, vp, vp, i64, i32, i32, vp, vp]
     L.mhc_sync_status.argtypes = [vp]
     L.mhc_set_path.argtypes = [i32]
+    L.xhc_conv_gs.argtypes = [vp, i32, vp, ct.POINTER(ct.c_int), i32, i64, i32, i64, vp, vp]
     L.mhc_set_wait_limit.argtypes = [ct.c_longlong]
-    for name in ("mhc_pre", "mhc_post", "mhc_sync_status", "mhc_set_path", "mhc_set_wait_limit"):
+    for name in ("mhc_pre", "mhc_post", "mhc_sync_status", "mhc_set_path", "mhc_set_wait_limit",
+                 "xhc_conv_gs"):
         getattr(L, name).restype = ct.c_int
     return L
 
@@ -145,3 +147,22 @@ def mhc_set_path(path: int) -> None:
 def mhc_set_wait_limit(polls: int) -> None:
     """Polls before a bounded on-device wait gives up (tests of the timeout path)."""
     _check(native().mhc_set_wait_limit(int(polls)))
+
+
+def xhc_conv_gs(F_out, conv_w, seq_len=None, *, V=None, stream=None):
+    """Causal depthwise convolutions + Gram-Schmidt (see include/mhc.h).
+    F_out [T][C]; conv_w: a list of r fp32 weight tensors [kappa_j][C] or one
+    concatenated tensor with `kappa` given as conv_w[1].  Returns V [T][r+1][C] fp32."""
+    if isinstance(conv_w, (list, tuple)) and all(hasattr(w, "shape") for w in conv_w):
+        kappa = [int(w.shape[0]) for w in conv_w]
+        wcat = torch.cat([w.reshape(-1) for w in conv_w]).contiguous()
+    else:
+        wcat, kappa = conv_w
+    T, C = F_out.shape
+    r = len(kappa)
+    if V is None:
+        V = torch.empty((T, r + 1, C), dtype=torch.float32, device=F_out.device)
+    ka = (ct.c_int * r)(*kappa)
+    _check(native().xhc_conv_gs(_ptr(F_out), _dt(F_out), _ptr(wcat), ka, r, T, C,
+                                int(seq_len or max(T, 1)), _ptr(V), _stream(stream)))
+    return V

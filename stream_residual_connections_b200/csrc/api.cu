@@ -149,6 +149,33 @@ mhc_status mhc_post(const void* X, const void* F_out, mhc_dtype dt, const float*
     return launch_post(X, F_out, dt, H_post, H_res, T, n, C, X_next, static_cast<cudaStream_t>(stream));
 }
 
+mhc_status xhc_conv_gs(const void* F_out, mhc_dtype dt, const float* conv_w, const int* kappa,
+                       int r, int64_t T, int C, int64_t seq_len, float* V, void* stream)
+{
+    const char* fn = "xhc_conv_gs";
+    g_msg[0] = 0;
+    REQUIRE(valid_dt(dt), MHC_ERR_INVALID_ARG, "%s: unknown dtype", fn);
+    REQUIRE(C > 0 && C % 8 == 0, MHC_ERR_INVALID_ARG, "%s: C=%d must be a positive multiple of 8", fn, C);
+    REQUIRE(T >= 0, MHC_ERR_INVALID_ARG, "%s: T=%lld < 0", fn, (long long)T);
+    REQUIRE(r >= 1 && r <= 4, MHC_ERR_INVALID_ARG, "%s: r=%d outside [1, 4]", fn, r);
+    REQUIRE(kappa != nullptr, MHC_ERR_INVALID_ARG, "%s: kappa (host int[r]) is NULL", fn);
+    int64_t wtot = 0;
+    for (int j = 0; j < r; ++j) {
+        REQUIRE(kappa[j] >= 1 && kappa[j] <= 64, MHC_ERR_INVALID_ARG, "%s: kappa[%d]=%d outside [1, 64]", fn, j, kappa[j]);
+        wtot += int64_t(kappa[j]) * C;
+    }
+    if (T == 0) return MHC_OK;
+    REQUIRE(seq_len >= 1, MHC_ERR_INVALID_ARG, "%s: seq_len=%lld < 1", fn, (long long)seq_len);
+    REQUIRE_PTR(F_out, "F_out");
+    REQUIRE_PTR(conv_w, "conv_w");
+    REQUIRE_PTR(V, "V");
+    const Range rV = range_of(V, size_t(T) * (r + 1) * C * 4);
+    REQUIRE(!overlap(rV, range_of(F_out, size_t(T) * C * dt_size(dt))) &&
+                !overlap(rV, range_of(conv_w, size_t(wtot) * 4)),
+            MHC_ERR_INVALID_ARG, "%s: V overlaps an input", fn);
+    return launch_conv_gs(F_out, dt, conv_w, kappa, r, T, C, seq_len, V, static_cast<cudaStream_t>(stream));
+}
+
 mhc_status mhc_set_path(mhc_path path)
 {
     g_msg[0] = 0;

@@ -28,6 +28,9 @@ mhc_status launch_pre_fma(const PreArgs& a, cudaStream_t s);
 bool pre_tc_supported(const PreArgs& a);
 mhc_status launch_pre_tc(const PreArgs& a, cudaStream_t s);
 
+mhc_status launch_conv_gs(const void* F, mhc_dtype dt, const float* W, const int* kappa, int r,
+                          int64_t T, int C, int64_t seq_len, float* V, cudaStream_t s);
+
 // Which mhc_pre path to take (MHC_PRE_PATH_*), process-wide.
 extern int g_pre_path;
 

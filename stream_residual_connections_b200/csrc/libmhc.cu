@@ -4,3 +4,4 @@
 #include "mhc_post.cu"
 #include "mhc_pre_fma.cu"
 #include "mhc_pre_tc.cu"
+#include "xhc_conv_gs.cu"
