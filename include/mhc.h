@@ -121,6 +121,36 @@ mhc_status mhc_post(const void* X, const void* F_out, mhc_dtype dt, const float*
 mhc_status xhc_conv_gs(const void* F_out, mhc_dtype dt, const float* conv_w, const int* kappa,
                        int r, int64_t T, int C, int64_t seq_len, float* V, void* stream);
 
+/*
+ * xhc_sparse_update -- sparse residual update and scatter of one xHC
+ * sublayer.  [xHC] "sparse residual stream architecture" (step 3) and
+ * "parameterisation": H_res and H_post are generated from the k active
+ * streams only; H_res is Sinkhorn-normalised (k x k), H_post = 2 sigma (k x Kr).
+ * For every token t, with X_act = rows idx[t][0..k-1] of X_t (slot order):
+ *   r = sqrt(sum(X_act^2)/(kC) + eps)
+ *   z = alpha * (vec(X_act) phi_act) / r + b_act   (alpha_act[0] on the k*k res
+ *       logits, alpha_act[1] on the k*Kr post logits)
+ *   H_res = Sinkhorn-Knopp(z[0:k*k] row-major, t_iters); H_post = 2 sigmoid(z[k*k:]) as [k][Kr]
+ *   X[t][idx[t][j]] = sum_l H_res[j][l] X_act[l] + w[t][j] * sum_q H_post[j][q] V[t][q]
+ * Streams not in idx[t] are not touched.
+ *
+ *   X       [T][N][C], dtype dt (read and written in place)
+ *   V       [T][Kr][C] fp32 (read; e.g. from xhc_conv_gs)
+ *   idx     [T][k] int32, distinct stream indices in [0, N) (e.g. from xhc_route);
+ *           a token with an entry outside [0, N) is left unchanged and
+ *           mhc_sync_status() then reports MHC_ERR_INVALID_ARG
+ *   w       [T][k] fp32 routing weights (read)
+ *   phi_act [k*k + k*Kr][k*C], dtype dt: the projection stored transposed
+ *           (row p = weights of logit p over vec(X_act)); rows res | post (read)
+ *   alpha_act HOST float[2] = (alpha_res, alpha_post);  b_act [k*k + k*Kr] fp32
+ *   H_res   [T][k][k] fp32, may be NULL;  H_post [T][k][Kr] fp32, may be NULL (written)
+ * This build: k <= 4, Kr <= 5, C % 64 == 0, N <= 64.
+ */
+mhc_status xhc_sparse_update(void* X, mhc_dtype dt, const float* V, int Kr, const int32_t* idx,
+                             const float* w, const void* phi_act, const float* alpha_act,
+                             const float* b_act, int64_t T, int N, int C, int k, int t_iters,
+                             float eps, float* H_res, float* H_post, void* stream);
+
 /* Kernel selection for the projection of mhc_pre. */
 typedef enum {
     MHC_PATH_AUTO = 0,    /* tensor cores where supported, else CUDA cores (default) */
@@ -148,9 +178,10 @@ mhc_status mhc_set_wait_limit(long long polls);
 
 /*
  * mhc_sync_status -- wait for `stream`, then report and clear the device-side
- * error word that bounded waits set when they expire: MHC_ERR_TIMEOUT if any
- * kernel of this library gave up waiting since the last call, else MHC_OK (or
- * MHC_ERR_CUDA if the stream itself failed).
+ * error word: MHC_ERR_TIMEOUT if a kernel of this library gave up a bounded
+ * wait since the last call, MHC_ERR_INVALID_ARG if a kernel met an
+ * out-of-range stream index in device data, else MHC_OK (or MHC_ERR_CUDA if
+ * the stream itself failed).
  */
 mhc_status mhc_sync_status(void* stream);
 

@@ -47,9 +47,11 @@ def _load():
     L.mhc_sync_status.argtypes = [vp]
     L.mhc_set_path.argtypes = [i32]
     L.xhc_conv_gs.argtypes = [vp, i32, vp, ct.POINTER(ct.c_int), i32, i64, i32, i64, vp, vp]
+    L.xhc_sparse_update.argtypes = [vp, i32, vp, i32, vp, vp, vp, fp, vp, i64, i32, i32, i32, i32,
+                                    f32, vp, vp, vp]
     L.mhc_set_wait_limit.argtypes = [ct.c_longlong]
     for name in ("mhc_pre", "mhc_post", "mhc_sync_status", "mhc_set_path", "mhc_set_wait_limit",
-                 "xhc_conv_gs"):
+                 "xhc_conv_gs", "xhc_sparse_update"):
         getattr(L, name).restype = ct.c_int
     return L
 
@@ -166,3 +168,21 @@ def xhc_conv_gs(F_out, conv_w, seq_len=None, *, V=None, stream=None):
     _check(native().xhc_conv_gs(_ptr(F_out), _dt(F_out), _ptr(wcat), ka, r, T, C,
                                 int(seq_len or max(T, 1)), _ptr(V), _stream(stream)))
     return V
+
+
+def xhc_sparse_update(X, V, idx, w, phi_act, alpha_act, b_act, t_iters: int = 20, eps: float = 1e-6,
+                      *, H_res=None, H_post=None, want_coeffs: bool = True, stream=None):
+    """Sparse k x k update + scatter, in place on X [T][N][C] (see include/mhc.h).
+    phi_act is [k*k + k*Kr][k*C] (transposed).  Returns (X, H_res, H_post)."""
+    T, N, C = X.shape
+    k = idx.shape[1]
+    Kr = V.shape[1]
+    if want_coeffs:
+        if H_res is None:
+            H_res = torch.empty((T, k, k), dtype=torch.float32, device=X.device)
+        if H_post is None:
+            H_post = torch.empty((T, k, Kr), dtype=torch.float32, device=X.device)
+    _check(native().xhc_sparse_update(_ptr(X), _dt(X), _ptr(V), Kr, _ptr(idx), _ptr(w), _ptr(phi_act),
+                                      _host3(alpha_act, 2), _ptr(b_act), T, N, C, k, int(t_iters),
+                                      float(eps), _ptr(H_res), _ptr(H_post), _stream(stream)))
+    return X, H_res, H_post

@@ -176,6 +176,50 @@ mhc_status xhc_conv_gs(const void* F_out, mhc_dtype dt, const float* conv_w, con
     return launch_conv_gs(F_out, dt, conv_w, kappa, r, T, C, seq_len, V, static_cast<cudaStream_t>(stream));
 }
 
+mhc_status xhc_sparse_update(void* X, mhc_dtype dt, const float* V, int Kr, const int32_t* idx,
+                             const float* w, const void* phi_act, const float* alpha_act,
+                             const float* b_act, int64_t T, int N, int C, int k, int t_iters,
+                             float eps, float* H_res, float* H_post, void* stream)
+{
+    const char* fn = "xhc_sparse_update";
+    g_msg[0] = 0;
+    REQUIRE(valid_dt(dt), MHC_ERR_INVALID_ARG, "%s: unknown dtype", fn);
+    REQUIRE(C > 0 && C % 8 == 0, MHC_ERR_INVALID_ARG, "%s: C=%d must be a positive multiple of 8", fn, C);
+    REQUIRE(T >= 0, MHC_ERR_INVALID_ARG, "%s: T=%lld < 0", fn, (long long)T);
+    REQUIRE(N >= 1 && N <= 64, MHC_ERR_INVALID_ARG, "%s: N=%d outside [1, 64]", fn, N);
+    REQUIRE(k >= 1 && k <= N, MHC_ERR_INVALID_ARG, "%s: k=%d outside [1, N]", fn, k);
+    REQUIRE(Kr >= 1, MHC_ERR_INVALID_ARG, "%s: Kr=%d < 1", fn, Kr);
+    REQUIRE(t_iters >= 0 && t_iters <= 1000, MHC_ERR_INVALID_ARG, "%s: t_iters=%d outside [0, 1000]", fn, t_iters);
+    REQUIRE(eps >= 0.0f, MHC_ERR_INVALID_ARG, "%s: eps < 0", fn);
+    REQUIRE(alpha_act != nullptr, MHC_ERR_INVALID_ARG, "%s: alpha_act (host float[2]) is NULL", fn);
+    REQUIRE(k <= 4 && Kr <= 5, MHC_ERR_UNSUPPORTED, "%s: k=%d, Kr=%d (this build: k <= 4, Kr <= 5)", fn, k, Kr);
+    REQUIRE(C % 64 == 0, MHC_ERR_UNSUPPORTED, "%s: C=%d must be a multiple of 64", fn, C);
+    if (T == 0) return MHC_OK;
+    REQUIRE_PTR(X, "X");
+    REQUIRE_PTR(V, "V");
+    REQUIRE(idx != nullptr && w != nullptr, MHC_ERR_INVALID_ARG, "%s: idx or w is NULL", fn);
+    REQUIRE_PTR(phi_act, "phi_act");
+    REQUIRE(b_act != nullptr, MHC_ERR_INVALID_ARG, "%s: b_act is NULL", fn);
+    const int Pa = k * k + k * Kr;
+    const size_t es = dt_size(dt);
+    const Range rX = range_of(X, size_t(T) * N * C * es);
+    const Range ins[5] = {range_of(V, size_t(T) * Kr * C * 4), range_of(idx, size_t(T) * k * 4),
+                          range_of(w, size_t(T) * k * 4), range_of(phi_act, size_t(Pa) * k * C * es),
+                          range_of(b_act, size_t(Pa) * 4)};
+    for (int i = 0; i < 5; ++i)
+        REQUIRE(!overlap(rX, ins[i]), MHC_ERR_INVALID_ARG, "%s: X overlaps an input", fn);
+    const Range outs[2] = {range_of(H_res, H_res ? size_t(T) * k * k * 4 : 0),
+                           range_of(H_post, H_post ? size_t(T) * k * Kr * 4 : 0)};
+    for (int o = 0; o < 2; ++o) {
+        REQUIRE(!overlap(outs[o], rX), MHC_ERR_INVALID_ARG, "%s: a coefficient output overlaps X", fn);
+        for (int i = 0; i < 5; ++i)
+            REQUIRE(!overlap(outs[o], ins[i]), MHC_ERR_INVALID_ARG, "%s: a coefficient output overlaps an input", fn);
+    }
+    UpdateArgs a{X, dt, V, Kr, idx, w, phi_act, {alpha_act[0], alpha_act[1]}, b_act, T, N, C, k,
+                 t_iters, eps, H_res, H_post};
+    return launch_sparse_update(a, static_cast<cudaStream_t>(stream));
+}
+
 mhc_status mhc_set_path(mhc_path path)
 {
     g_msg[0] = 0;
@@ -204,8 +248,13 @@ mhc_status mhc_sync_status(void* stream)
         const unsigned int zero = 0;
         e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
         if (e != cudaSuccess) return cuda_status(e, "mhc_sync_status: clear error word");
-        set_error("a bounded on-device wait expired (error word 0x%x)", flag);
-        return MHC_ERR_TIMEOUT;
+        if (flag & 1u) {
+            set_error("a bounded on-device wait expired (error word 0x%x)", flag);
+            return MHC_ERR_TIMEOUT;
+        }
+        set_error("a kernel met an out-of-range stream index; those tokens were left unchanged "
+                  "(error word 0x%x)", flag);
+        return MHC_ERR_INVALID_ARG;
     }
     return MHC_OK;
 }

@@ -31,6 +31,14 @@ mhc_status launch_pre_tc(const PreArgs& a, cudaStream_t s);
 mhc_status launch_conv_gs(const void* F, mhc_dtype dt, const float* W, const int* kappa, int r,
                           int64_t T, int C, int64_t seq_len, float* V, cudaStream_t s);
 
+struct UpdateArgs {
+    void* X; mhc_dtype dt; const float* V; int Kr; const int32_t* idx; const float* w;
+    const void* phi; float alpha[2]; const float* b;
+    int64_t T; int N; int C; int k; int t_iters; float eps;
+    float* H_res; float* H_post;
+};
+mhc_status launch_sparse_update(const UpdateArgs& a, cudaStream_t s);
+
 // Which mhc_pre path to take (MHC_PRE_PATH_*), process-wide.
 extern int g_pre_path;
 

@@ -5,3 +5,4 @@
 #include "mhc_pre_fma.cu"
 #include "mhc_pre_tc.cu"
 #include "xhc_conv_gs.cu"
+#include "xhc_update.cu"

@@ -9,7 +9,7 @@
 //
 // Warp roles (16 warps):
 //   0      TMA producer: X[tile, stream i, 64-channel block] boxes (Mt rows x
-//          128 B, 128-byte swizzle, L2 evict-last) through an 8-stage ring;
+//          128 B, 128-byte swizzle, L2 evict-last) through a 14-stage ring;
 //          it runs at most LAG tiles ahead of the x_in warps, which keeps the
 //          x_in re-read inside L2.
 //   1      MMA issuer: D[128 x NB] += X_chunk[128 x 64] * phiT_chunk[NB x 64]^T
@@ -17,10 +17,13 @@
 //          across tiles; rows >= Mt are never read).
 //   2-3    sum of squares of every tile row of every ring stage (Eq.15),
 //          handed to the epilogue through a double-buffered shared array.
-//   4-5    epilogue: partial logits from TMEM; exchange of the 8 partial
-//          (logits, sum of squares) rows through DSMEM; coefficients of 8
-//          tokens per CTA (Eq.16-19; a row-parallel Sinkhorn over 8 lanes);
-//          H_pre broadcast to the cluster through DSMEM.
+//   4-5    epilogue: each tile row's partial (logits, sum of squares) from TMEM
+//          is pushed with st.async into the shared memory of the CTA that owns
+//          the token (8 tokens per CTA); the owner reduces the 8 partial rows,
+//          computes the coefficients (Eq.16-19; row-parallel Sinkhorn over 8
+//          lanes) and pushes H_pre to every CTA of the cluster.  The pushes
+//          complete transactions on the receivers' mbarriers, so no fence or
+//          remote arrive sits on this path.
 //   6-15   x_in = H_pre X for this CTA's channels, re-reading the tile's X
 //          slice from L2 (evict-first on this last read).
 // The roles meet only through mbarriers and one progress counter, so the TMA
@@ -44,7 +47,7 @@ constexpr int MROWS = 128;       // MMA M (TMEM lanes); a tile uses the first Mt
 constexpr int MT_CAP = 64;       // token rows per tile: bounds the L2 footprint of the x_in re-read
 constexpr int KC = 64;           // K elements per chunk (one 128-byte row)
 constexpr int STAGE_BYTES = MT_CAP * 128;
-constexpr int STAGES = 8;
+constexpr int STAGES = 14;
 constexpr int NTHREADS = 512;
 constexpr int SS_WARP0 = 2, SS_WARPS = 2;                  // one tile row per thread
 constexpr int EPI_WARP0 = 4, EPI_WARPS = 2, EPI_THREADS = 64;
@@ -65,7 +68,7 @@ template <int N> struct Cfg {
 
 enum Bar { B_FULL = 0, B_EMPTY = B_FULL + STAGES, B_TFULL = B_EMPTY + STAGES, B_TEMPTY = B_TFULL + 2,
            B_SSFULL = B_TEMPTY + 2, B_SSEMPTY = B_SSFULL + 2, B_PART = B_SSEMPTY + 2, B_HPRE,
-           B_EPI, B_XIN, B_PHI, B_DRAIN, B_COUNT };
+           B_XIN = B_HPRE + 2, B_PHI, B_DRAIN, B_COUNT };
 
 struct Layout {
     uint32_t phi, ring, part, ss, hpre, bars, slot, total;
@@ -78,7 +81,7 @@ __host__ __device__ inline Layout layout_for(int NQ) {
     L.phi = 0;
     L.ring = uint32_t(NQ) * G::R * 128;                      // multiple of 1024
     L.part = L.ring + STAGES * STAGE_BYTES;
-    L.ss = L.part + MT_CAP * G::PSP * 4;
+    L.ss = L.part + CL * TOK_PER_CTA * G::PSP * 4;         // [source CTA][token][PSP]
     L.hpre = L.ss + 2 * MT_CAP * 4;
     L.bars = (L.hpre + 2 * MT_CAP * N * 4 + 15) / 16 * 16;
     L.slot = L.bars + B_COUNT * 8;
@@ -111,7 +114,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     const Layout L = layout_for<N>(NQ);
     uint8_t* sphi = smem + L.phi;
     uint8_t* sring = smem + L.ring;
-    float* spart = reinterpret_cast<float*>(smem + L.part);
+    float* rpart = reinterpret_cast<float*>(smem + L.part);   // [CL][TOK_PER_CTA][PSP], pushed by the cluster
     float* sss = reinterpret_cast<float*>(smem + L.ss);       // [2][MT_CAP]
     float* shpre = reinterpret_cast<float*>(smem + L.hpre);   // [2][MT_CAP][N]
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
@@ -121,9 +124,8 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     uint64_t* tempty = bars + B_TEMPTY;
     uint64_t* ssfull = bars + B_SSFULL;
     uint64_t* ssempty = bars + B_SSEMPTY;
-    uint64_t* part_ready = bars + B_PART;
-    uint64_t* hpre_ready = bars + B_HPRE;
-    uint64_t* epi_sync = bars + B_EPI;
+    uint64_t* part_full = bars + B_PART;     // this CTA's tokens: all CL partial rows landed
+    uint64_t* hpre_full = bars + B_HPRE;     // [2] H_pre of every tile row landed (per tile parity)
     uint64_t* xin_prog = bars + B_XIN;
     uint64_t* phi_full = bars + B_PHI;
     uint64_t* drain = bars + B_DRAIN;
@@ -150,9 +152,11 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             mbar_init(&ssfull[a], SS_WARPS);
             mbar_init(&ssempty[a], EPI_WARPS);
         }
-        mbar_init(part_ready, CL);
-        mbar_init(hpre_ready, CL);
-        mbar_init(epi_sync, EPI_THREADS);
+        // one local arrival (with the expected byte count) per phase; the bytes
+        // come from st.async pushes of the cluster
+        mbar_init(part_full, 1);
+        mbar_init(&hpre_full[0], 1);
+        mbar_init(&hpre_full[1], 1);
         mbar_init(xin_prog, XIN_WARPS);
         mbar_init(phi_full, 1);
         mbar_init(drain, 1);
@@ -285,11 +289,22 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         const int qd = warp & 3;                        // TMEM lane quarter of this warp (0, 1)
         const int m = qd * 32 + lane;                   // token row within the tile
         const float inv_K = 1.0f / float(N * C);
+        constexpr uint32_t PART_BYTES = CL * TOK_PER_CTA * PSP * 4;
+        constexpr uint32_t HPRE_BYTES = MT_CAP * N * 4;
+        // the partial row of tile row m goes to its owner CTA m / TOK_PER_CTA, slot (rank, m % TOK_PER_CTA)
+        const uint32_t owner = uint32_t(m / TOK_PER_CTA);
+        const uint32_t push_dst = mapa(smem_u32(rpart + (int(rank) * TOK_PER_CTA + m % TOK_PER_CTA) * PSP), owner);
+        const uint32_t push_bar = mapa(smem_u32(part_full), owner);
         int it = 0;
         for (int tile = cluster_id; tile < num_tiles; tile += nclusters, ++it) {
             const int64_t t0 = int64_t(tile) * Mt;
             const int acc = it & 1;
             const uint32_t par = uint32_t((it >> 1) & 1);
+            if (et == 0) {
+                // expected bytes of this tile's phases; pushes may land before or after
+                mbar_arrive_expect_tx(part_full, PART_BYTES);
+                mbar_arrive_expect_tx(&hpre_full[acc], HPRE_BYTES);
+            }
             if (!mbar_wait(&tfull[acc], par) || !mbar_wait(&ssfull[acc], par)) { s_abort = 1; break; }
             tc_fence_after();
             float d[NB];
@@ -307,8 +322,10 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             __syncwarp();
             if (lane == 0) { mbar_arrive(&tempty[acc]); mbar_arrive(&ssempty[acc]); }
 
-            // share this CTA's partial logits and sum of squares with the cluster
-            float* prow = spart + m * PSP;
+            // H_pre of tile it lands in buffer it&1, last read by the x_in warps for
+            // tile it-2: they must have moved on (they arrive after their tile it-1 wait)
+            if (it >= 1 && !mbar_wait(xin_prog, uint32_t((it - 1) & 1))) { s_abort = 1; break; }
+            // push (partial logits, sum of squares) of row m to its owner
 #pragma unroll
             for (int p = 0; p < PSP; p += 4) {
                 float4 w4;
@@ -316,30 +333,21 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 w4.y = p + 1 < P ? d[p + 1] : (p + 1 == P ? ss : 0.0f);
                 w4.z = p + 2 < P ? d[p + 2] : (p + 2 == P ? ss : 0.0f);
                 w4.w = p + 3 < P ? d[p + 3] : (p + 3 == P ? ss : 0.0f);
-                *reinterpret_cast<float4*>(prow + p) = w4;
+                st_async_f32x4(push_dst + p * 4, w4, push_bar);
             }
-            asm volatile("fence.acq_rel.cluster;" ::: "memory");
-            mbar_arrive(epi_sync);
-            if (et == 0) {
-                bool ok = mbar_wait(epi_sync, 0);
-                // the x_in warps have moved past tile it-1, so its H_pre buffer may be rewritten
-                if (ok && it >= 1) ok = mbar_wait(xin_prog, uint32_t((it - 1) & 1));
-                if (!ok) { s_abort = 1; break; }
-                for (uint32_t r = 0; r < CL; ++r) mbar_arrive_cluster(mapa(smem_u32(part_ready), r));
-            }
-            if (!mbar_wait<true>(part_ready, uint32_t(it & 1))) { s_abort = 1; break; }
+            if (!mbar_wait(part_full, uint32_t(it & 1))) { s_abort = 1; break; }
 
-            // Coefficients of TOK_PER_CTA tokens: a group of 8 lanes per token; lane g
-            // fetches the partial row of CTA g, the group reduces, then lane g < N
-            // carries row g of H_res through a row-parallel Sinkhorn.
+            // Coefficients of this CTA's TOK_PER_CTA tokens: a group of 8 lanes per
+            // token; lane g takes the partial row from CTA g, the group reduces, then
+            // lane g < N carries row g of H_res through a row-parallel Sinkhorn.
             {
                 const int jj = et >> 3, g = et & 7;
                 const int j = int(rank) * TOK_PER_CTA + jj;     // row within the tile
-                const uint32_t pbase = mapa(smem_u32(spart + j * PSP), uint32_t(g));
+                const float* src = rpart + (g * TOK_PER_CTA + jj) * PSP;
                 float v[PSP];
 #pragma unroll
                 for (int p = 0; p < PSP; p += 4) {
-                    const float4 f4 = ld_cluster_f32x4(pbase + p * 4);
+                    const float4 f4 = *reinterpret_cast<const float4*>(src + p);
                     v[p] = f4.x; v[p + 1] = f4.y; v[p + 2] = f4.z; v[p + 3] = f4.w;
                 }
 #pragma unroll
@@ -363,25 +371,24 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                             row[k] = a2 * v[2 * N + i * N + k] * inv_r + __ldg(b + 2 * N + i * N + k);
                     }
                 sinkhorn_group8<N>(row, g, t_iters);                               // Eq.(19)
-                const int64_t t = t0 + j;
-                if (g < N && jj < TOK_PER_CTA && j < Mt && t < T) {
+                if (g < N) {
                     const float hp = sigmoidf_(zpre);                              // Eq.(17)
-                    Hpost[t * N + g] = 2.0f * sigmoidf_(zpost);                    // Eq.(18)
-                    if (Hpre) Hpre[t * N + g] = hp;
-#pragma unroll
-                    for (int k = 0; k < N; ++k) Hres[(t * N + g) * N + k] = row[k];
+                    // every CTA needs H_pre of every tile row for its x_in channels
                     const uint32_t hoff = smem_u32(shpre + (acc * MT_CAP + j) * N + g);
-                    for (uint32_t rr = 0; rr < CL; ++rr) st_cluster_f32(mapa(hoff, rr), hp);
+                    const uint32_t hbar = smem_u32(&hpre_full[acc]);
+                    for (uint32_t rr = 0; rr < CL; ++rr) st_async_f32(mapa(hoff, rr), hp, mapa(hbar, rr));
+                    const int64_t t = t0 + j;
+                    if (j < Mt && t < T) {
+                        Hpost[t * N + g] = 2.0f * sigmoidf_(zpost);                // Eq.(18)
+                        if (Hpre) Hpre[t * N + g] = hp;
+#pragma unroll
+                        for (int k = 0; k < N; ++k) Hres[(t * N + g) * N + k] = row[k];
+                    }
                 }
             }
-            asm volatile("fence.acq_rel.cluster;" ::: "memory");
-            mbar_arrive(epi_sync);
-            if (et == 0) {
-                if (!mbar_wait(epi_sync, 1)) { s_abort = 1; break; }
-                for (uint32_t r = 0; r < CL; ++r) mbar_arrive_cluster(mapa(smem_u32(hpre_ready), r));
-            }
-            // the partial rows of this tile are no longer read once every CTA has its H_pre
-            if (!mbar_wait<true>(hpre_ready, uint32_t(it & 1))) { s_abort = 1; break; }
+            // every owner has read its partial rows of this tile once this CTA holds the
+            // tile's H_pre; only then may the next tile's partial rows be pushed
+            if (!mbar_wait(&hpre_full[acc], par)) { s_abort = 1; break; }
         }
     } else {
         // ------------------------------------------------------------ x_in
@@ -390,7 +397,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         const int VPT = Cs / 8;                          // 16-byte vectors per token
         int it = 0;
         for (int tile = cluster_id; tile < num_tiles; tile += nclusters, ++it) {
-            if (!mbar_wait<true>(hpre_ready, uint32_t(it & 1))) { s_abort = 1; break; }
+            if (!mbar_wait(&hpre_full[it & 1], uint32_t((it >> 1) & 1))) { s_abort = 1; break; }
             __syncwarp();
             if (lane == 0) mbar_arrive(xin_prog);
             const int64_t t0 = int64_t(tile) * Mt;

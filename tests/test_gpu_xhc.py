@@ -71,3 +71,73 @@ def test_conv_gs_xhc_workload_sampled():
         ref = oracle.xhc_gs(Fw[-1:], G[-1:])[0]
         _check_V(V[t][None], ref[None], f"V[{t}]")
     assert np.isfinite(V).all()
+
+
+def _route_ref(inp):
+    return oracle.xhc_route(inp["X"], inp["phi_read"], inp["alpha_read"], inp["b_read"], inp["k"], inp["m"])
+
+
+def _update_case(inp, tokens=None):
+    """GPU sparse update on inputs whose idx, w and V come from the oracle; compares
+    (all of, or the sampled `tokens` of) X_new, H_res, H_post."""
+    from tests.parity import check_coeffs, check_mix
+    T, N, C, k = inp["T"], inp["N"], inp["C"], inp["k"]
+    rt = _route_ref(inp)
+    V32 = oracle.xhc_conv_gs(inp["F"], inp["conv_w"]).astype(np.float32)
+    w32 = rt["w"].astype(np.float32)
+    Xd = dev(inp["X"])
+    phiT = dev(np.ascontiguousarray(inp["phi_act"].T))
+    _, Hr, Hp = M.xhc_sparse_update(Xd, torch.from_numpy(V32).cuda(), torch.from_numpy(rt["idx"]).cuda(),
+                                    torch.from_numpy(w32).cuda(), phiT, inp["alpha_act"],
+                                    torch.from_numpy(inp["b_act"]).cuda(), inp["t_iters"], inp["eps"])
+    M.mhc_sync_status()
+    sel = slice(None) if tokens is None else tokens
+    X0 = oracle.widen(inp["X"][sel])
+    ref, hr, hp = oracle.xhc_sparse_update(X0, V32[sel], rt["idx"][sel], w32[sel], inp["phi_act"],
+                                          inp["alpha_act"], inp["b_act"], inp["t_iters"], inp["eps"])
+    got = host(Xd)[sel]
+    check_coeffs(host(Hr)[sel], hr, "H_res")
+    check_coeffs(host(Hp)[sel], hp, "H_post")
+    idx = rt["idx"][sel]
+    for t in range(got.shape[0]):
+        inactive = sorted(set(range(N)) - set(idx[t].tolist()))
+        np.testing.assert_array_equal(got[t, inactive], X0[t, inactive])
+        act = idx[t]
+        absterms = (np.abs(X0[t, act]).sum(0)[None, :]
+                    + np.abs(w32[sel][t])[:, None] * np.abs(V32[sel][t]).sum(0)[None, :])
+        check_mix(got[t, act], ref[t, act], absterms, inp["dtype"], f"X_new[{t}]")
+
+
+@pytest.mark.parametrize("T,N,k,m,C,dtype", [(37, 8, 4, 2, 128, "bf16"), (50, 6, 3, 1, 192, "f32"),
+                                             (33, 16, 4, 2, 256, "bf16"), (20, 4, 2, 1, 64, "bf16")])
+def test_sparse_update_matches_oracle(T, N, k, m, C, dtype):
+    inp = synth.xhc_inputs(T, N=N, k=k, m=m, C=C, dtype=dtype, seed=600 + T + N)
+    _update_case(inp)
+
+
+def test_sparse_update_out_of_range_index_is_reported_and_token_untouched():
+    T, N, k, C = 8, 8, 4, 64
+    inp = synth.xhc_inputs(T, N=N, k=k, m=2, C=C, seed=7)
+    idx = np.tile(np.array([0, 1, 2, 3], dtype=np.int32), (T, 1))
+    idx[3, 2] = N + 5
+    Xd = dev(inp["X"])
+    X0 = host(Xd)
+    V = torch.zeros((T, 4, C), device="cuda")
+    M.xhc_sparse_update(Xd, V, torch.from_numpy(idx).cuda(), torch.ones((T, k), device="cuda"),
+                        dev(np.ascontiguousarray(inp["phi_act"].T)), inp["alpha_act"],
+                        torch.from_numpy(inp["b_act"]).cuda())
+    with pytest.raises(M.MhcError) as e:
+        M.mhc_sync_status()
+    assert e.value.status == M.MHC_ERR_INVALID_ARG
+    got = host(Xd)
+    np.testing.assert_array_equal(got[3], X0[3])
+    assert not np.array_equal(got[2], X0[2])
+    M.mhc_sync_status()
+
+
+def test_sparse_update_xhc_workload_sampled():
+    """T=8192, N=16, k=4 (m=2), C=2048: the update runs on all tokens; 48 are compared."""
+    inp = synth.xhc_inputs(**synth.WORKLOADS["xhc"])
+    rng = np.random.default_rng(2)
+    toks = np.unique(np.concatenate([[0, 8191], rng.choice(8192, 46, replace=False)]))
+    _update_case(inp, toks)
