@@ -103,6 +103,32 @@ mhc_status mhc_post(const void* X, const void* F_out, mhc_dtype dt, const float*
                     const float* H_res, int64_t T, int n, int C, void* X_next, void* stream);
 
 /*
+ * xhc_route -- stream routing and dense read of one xHC sublayer.
+ * [xHC] "sparse residual stream architecture", steps 1 (routing: m fixed
+ * streams with weight 1, k-m chosen by TopK over sigmoid scores derived from
+ * the full N-stream state) and 2 (dense read over all N streams);
+ * "parameterisation" (gated projection, alpha and bias).  For every token t:
+ *   x = vec(X_t) (N*C); r = sqrt(sum(x^2)/(NC) + eps)
+ *   z = alpha_seg * (x phi_read) / r + b_read      (R = 2N - m logits)
+ *   H_pre[i] = sigmoid(z[i]), i < N;  score[s-m] = sigmoid(z[N + s - m]), s = m..N-1
+ *   active = {0..m-1} and the k-m streams s >= m with the highest score (an exact
+ *            tie goes to the lower index); idx[t] lists them in ascending order;
+ *            w = 1 for fixed streams, the score for routed ones
+ *   x_in[c] = sum_{i<N} H_pre[i] * X_t[i][c]
+ *
+ *   X        [T][N][C], dtype dt (read)
+ *   phi_read [R][N*C], dtype dt: the router projection stored transposed; rows
+ *            0..N-1 give the H_pre logits, rows N..R-1 the route logits (read)
+ *   alpha_read HOST float[2] = (alpha_pre, alpha_route);  b_read [R] fp32 (read)
+ *   x_in [T][C] dtype dt; H_pre [T][N] fp32 (may be NULL); score [T][N-m] fp32
+ *   (may be NULL); idx [T][k] int32; w [T][k] fp32 (written)
+ * N <= 32, 0 <= m <= k <= N.
+ */
+mhc_status xhc_route(const void* X, mhc_dtype dt, const void* phi_read, const float* alpha_read,
+                     const float* b_read, int64_t T, int N, int C, int k, int m, float eps, void* x_in,
+                     float* H_pre, float* score, int32_t* idx, float* w, void* stream);
+
+/*
  * xhc_conv_gs -- temporal feature augmentation of the xHC write-back.
  * [xHC] "temporal feature augmentation": r causal depthwise convolutions of
  * the sublayer output and Gram-Schmidt orthogonalisation of the Kr = r + 1

@@ -46,12 +46,13 @@ def _load():
     L.mhc_post.argtypes = [vp, vp, i32, vp, vp, i64, i32, i32, vp, vp]
     L.mhc_sync_status.argtypes = [vp]
     L.mhc_set_path.argtypes = [i32]
+    L.xhc_route.argtypes = [vp, i32, vp, fp, vp, i64, i32, i32, i32, i32, f32, vp, vp, vp, vp, vp, vp]
     L.xhc_conv_gs.argtypes = [vp, i32, vp, ct.POINTER(ct.c_int), i32, i64, i32, i64, vp, vp]
     L.xhc_sparse_update.argtypes = [vp, i32, vp, i32, vp, vp, vp, fp, vp, i64, i32, i32, i32, i32,
                                     f32, vp, vp, vp]
     L.mhc_set_wait_limit.argtypes = [ct.c_longlong]
     for name in ("mhc_pre", "mhc_post", "mhc_sync_status", "mhc_set_path", "mhc_set_wait_limit",
-                 "xhc_conv_gs", "xhc_sparse_update"):
+                 "xhc_conv_gs", "xhc_sparse_update", "xhc_route"):
         getattr(L, name).restype = ct.c_int
     return L
 
@@ -186,3 +187,26 @@ def xhc_sparse_update(X, V, idx, w, phi_act, alpha_act, b_act, t_iters: int = 20
                                       _host3(alpha_act, 2), _ptr(b_act), T, N, C, k, int(t_iters),
                                       float(eps), _ptr(H_res), _ptr(H_post), _stream(stream)))
     return X, H_res, H_post
+
+
+def xhc_route(X, phi_read, alpha_read, b_read, k: int, m: int, eps: float = 1e-6, *, x_in=None,
+              H_pre=None, score=None, idx=None, w=None, want_scores: bool = True, stream=None):
+    """Routing + dense read (see include/mhc.h).  X [T][N][C]; phi_read [2N-m][N*C]
+    (transposed).  Returns (x_in, H_pre, score, idx, w)."""
+    T, N, C = X.shape
+    dev = X.device
+    if x_in is None:
+        x_in = torch.empty((T, C), dtype=X.dtype, device=dev)
+    if want_scores:
+        if H_pre is None:
+            H_pre = torch.empty((T, N), dtype=torch.float32, device=dev)
+        if score is None:
+            score = torch.empty((T, max(N - m, 1)), dtype=torch.float32, device=dev)
+    if idx is None:
+        idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    if w is None:
+        w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    _check(native().xhc_route(_ptr(X), _dt(X), _ptr(phi_read), _host3(alpha_read, 2), _ptr(b_read), T, N,
+                              C, int(k), int(m), float(eps), _ptr(x_in), _ptr(H_pre), _ptr(score),
+                              _ptr(idx), _ptr(w), _stream(stream)))
+    return x_in, H_pre, score, idx, w

@@ -149,6 +149,43 @@ mhc_status mhc_post(const void* X, const void* F_out, mhc_dtype dt, const float*
     return launch_post(X, F_out, dt, H_post, H_res, T, n, C, X_next, static_cast<cudaStream_t>(stream));
 }
 
+mhc_status xhc_route(const void* X, mhc_dtype dt, const void* phi_read, const float* alpha_read,
+                     const float* b_read, int64_t T, int N, int C, int k, int m, float eps, void* x_in,
+                     float* H_pre, float* score, int32_t* idx, float* w, void* stream)
+{
+    const char* fn = "xhc_route";
+    g_msg[0] = 0;
+    REQUIRE(valid_dt(dt), MHC_ERR_INVALID_ARG, "%s: unknown dtype", fn);
+    REQUIRE(C > 0 && C % 8 == 0, MHC_ERR_INVALID_ARG, "%s: C=%d must be a positive multiple of 8", fn, C);
+    REQUIRE(T >= 0, MHC_ERR_INVALID_ARG, "%s: T=%lld < 0", fn, (long long)T);
+    REQUIRE(N >= 1 && N <= 32, MHC_ERR_INVALID_ARG, "%s: N=%d outside [1, 32]", fn, N);
+    REQUIRE(m >= 0 && m <= k && k <= N, MHC_ERR_INVALID_ARG, "%s: need 0 <= m <= k <= N (k=%d, m=%d)", fn, k, m);
+    REQUIRE(eps >= 0.0f, MHC_ERR_INVALID_ARG, "%s: eps < 0", fn);
+    REQUIRE(alpha_read != nullptr, MHC_ERR_INVALID_ARG, "%s: alpha_read (host float[2]) is NULL", fn);
+    if (T == 0) return MHC_OK;
+    REQUIRE_PTR(X, "X");
+    REQUIRE_PTR(phi_read, "phi_read");
+    REQUIRE(b_read != nullptr, MHC_ERR_INVALID_ARG, "%s: b_read is NULL", fn);
+    REQUIRE_PTR(x_in, "x_in");
+    REQUIRE(idx != nullptr && w != nullptr, MHC_ERR_INVALID_ARG, "%s: idx or w is NULL", fn);
+    const int R = 2 * N - m;
+    const size_t es = dt_size(dt);
+    const Range ins[3] = {range_of(X, size_t(T) * N * C * es), range_of(phi_read, size_t(R) * N * C * es),
+                          range_of(b_read, size_t(R) * 4)};
+    const Range outs[5] = {range_of(x_in, size_t(T) * C * es), range_of(H_pre, H_pre ? size_t(T) * N * 4 : 0),
+                           range_of(score, score ? size_t(T) * (N - m) * 4 : 0), range_of(idx, size_t(T) * k * 4),
+                           range_of(w, size_t(T) * k * 4)};
+    for (int o = 0; o < 5; ++o) {
+        for (int i = 0; i < 3; ++i)
+            REQUIRE(!overlap(outs[o], ins[i]), MHC_ERR_INVALID_ARG, "%s: an output overlaps an input", fn);
+        for (int q = 0; q < o; ++q)
+            REQUIRE(!overlap(outs[o], outs[q]), MHC_ERR_INVALID_ARG, "%s: outputs overlap", fn);
+    }
+    RouteArgs a{X, dt, phi_read, {alpha_read[0], alpha_read[1]}, b_read, T, N, C, k, m, eps, x_in, H_pre,
+                score, idx, w};
+    return launch_route(a, static_cast<cudaStream_t>(stream));
+}
+
 mhc_status xhc_conv_gs(const void* F_out, mhc_dtype dt, const float* conv_w, const int* kappa,
                        int r, int64_t T, int C, int64_t seq_len, float* V, void* stream)
 {

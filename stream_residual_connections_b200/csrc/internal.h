@@ -39,6 +39,13 @@ struct UpdateArgs {
 };
 mhc_status launch_sparse_update(const UpdateArgs& a, cudaStream_t s);
 
+struct RouteArgs {
+    const void* X; mhc_dtype dt; const void* phi; float alpha[2]; const float* b;
+    int64_t T; int N; int C; int k; int m; float eps;
+    void* x_in; float* H_pre; float* score; int32_t* idx; float* w;
+};
+mhc_status launch_route(const RouteArgs& a, cudaStream_t s);
+
 // Which mhc_pre path to take (MHC_PRE_PATH_*), process-wide.
 extern int g_pre_path;
 

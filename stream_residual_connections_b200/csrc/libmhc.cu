@@ -6,3 +6,4 @@
 #include "mhc_pre_tc.cu"
 #include "xhc_conv_gs.cu"
 #include "xhc_update.cu"
+#include "xhc_route.cu"

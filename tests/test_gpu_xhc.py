@@ -77,12 +77,12 @@ def _route_ref(inp):
     return oracle.xhc_route(inp["X"], inp["phi_read"], inp["alpha_read"], inp["b_read"], inp["k"], inp["m"])
 
 
-def _update_case(inp, tokens=None):
+def _update_case(inp, tokens=None, rt=None):
     """GPU sparse update on inputs whose idx, w and V come from the oracle; compares
     (all of, or the sampled `tokens` of) X_new, H_res, H_post."""
     from tests.parity import check_coeffs, check_mix
     T, N, C, k = inp["T"], inp["N"], inp["C"], inp["k"]
-    rt = _route_ref(inp)
+    rt = _route_ref(inp) if rt is None else rt
     V32 = oracle.xhc_conv_gs(inp["F"], inp["conv_w"]).astype(np.float32)
     w32 = rt["w"].astype(np.float32)
     Xd = dev(inp["X"])
@@ -137,7 +137,93 @@ def test_sparse_update_out_of_range_index_is_reported_and_token_untouched():
 
 def test_sparse_update_xhc_workload_sampled():
     """T=8192, N=16, k=4 (m=2), C=2048: the update runs on all tokens; 48 are compared."""
-    inp = synth.xhc_inputs(**synth.WORKLOADS["xhc"])
+    inp, rt = xhc_full()
     rng = np.random.default_rng(2)
     toks = np.unique(np.concatenate([[0, 8191], rng.choice(8192, 46, replace=False)]))
-    _update_case(inp, toks)
+    _update_case(inp, toks, rt)
+
+
+def gapped(inp, gap=1e-4, max_rounds=30, with_route=False):
+    """Redraw (from derived seeds) the X rows of tokens whose routed-score gap
+    between the (k-m)-th and (k-m+1)-th highest score is <= gap (fp64 oracle),
+    so that every TopK selection is decided well above rounding.  With
+    with_route, also return the oracle's routing of the final inputs."""
+    k, m, N = inp["k"], inp["m"], inp["N"]
+    rows = np.arange(inp["T"])
+    full = None
+    for attempt in range(max_rounds + 1):
+        out = oracle.xhc_route(inp["X"][rows], inp["phi_read"], inp["alpha_read"], inp["b_read"], k, m,
+                               inp["eps"])
+        if full is None:
+            full = out
+        else:
+            for key in full:
+                full[key][rows] = out[key]
+        sc = out["score"]
+        if k == m or k - m >= sc.shape[1]:
+            break
+        s = -np.sort(-sc, axis=1)
+        bad = rows[(s[:, k - m - 1] - s[:, k - m]) <= gap]
+        if bad.size == 0:
+            break
+        assert attempt < max_rounds, "could not separate the routing scores"
+        synth.redraw_rows(inp["X"], bad, inp["seed"], attempt, inp["dtype"])
+        rows = bad
+    return (inp, full) if with_route else inp
+
+
+_FULL = {}
+
+
+def xhc_full():
+    """The T=8192, N=16, k=4, m=2, C=2048 workload with separated scores, and its
+    oracle routing (computed once per test session)."""
+    if "v" not in _FULL:
+        _FULL["v"] = gapped(synth.xhc_inputs(**synth.WORKLOADS["xhc"]), with_route=True)
+    return _FULL["v"]
+
+
+def _route_check(inp, tokens=None):
+    from tests.parity import check_coeffs, check_mix
+    k, m = inp["k"], inp["m"]
+    x_in, Hp, sc, idx, w = M.xhc_route(dev(inp["X"]), dev(np.ascontiguousarray(inp["phi_read"].T)),
+                                        inp["alpha_read"], torch.from_numpy(inp["b_read"]).cuda(), k, m,
+                                        inp["eps"])
+    torch.cuda.synchronize()
+    sel = slice(None) if tokens is None else tokens
+    ref = oracle.xhc_route(inp["X"][sel], inp["phi_read"], inp["alpha_read"], inp["b_read"], k, m, inp["eps"])
+    np.testing.assert_array_equal(idx.cpu().numpy()[sel], ref["idx"])
+    check_coeffs(host(Hp)[sel], ref["H_pre"], "H_pre")
+    check_coeffs(host(sc)[sel], ref["score"], "score")
+    check_coeffs(host(w)[sel], ref["w"], "w")
+    X = oracle.widen(inp["X"][sel])
+    check_mix(host(x_in)[sel], ref["x_in"], np.abs(X).sum(1), inp["dtype"], "x_in")
+
+
+@pytest.mark.parametrize("T,N,k,m,C,dtype", [(41, 8, 4, 2, 128, "bf16"), (30, 16, 4, 2, 264, "bf16"),
+                                             (25, 6, 3, 1, 64, "f32"), (20, 32, 8, 3, 64, "bf16"),
+                                             (17, 5, 5, 2, 32, "bf16"), (16, 4, 2, 0, 64, "f32")])
+def test_route_matches_oracle(T, N, k, m, C, dtype):
+    inp = gapped(synth.xhc_inputs(T, N=N, k=k, m=m, C=C, dtype=dtype, seed=700 + T + N))
+    _route_check(inp)
+
+
+def test_route_ties_go_to_the_lower_index():
+    T, N, k, m, C = 8, 8, 5, 2, 64
+    inp = synth.xhc_inputs(T, N=N, k=k, m=m, C=C, seed=9)
+    b = inp["b_read"].copy()
+    b[N:] = 0.0                                          # every routed score sigma(0)
+    _, _, sc, idx, w = M.xhc_route(dev(inp["X"]), dev(np.ascontiguousarray(inp["phi_read"].T)),
+                                   [0.0, 0.0], torch.from_numpy(b).cuda(), k, m)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(idx.cpu().numpy(), np.tile(np.arange(k, dtype=np.int32), (T, 1)))
+    np.testing.assert_allclose(w.cpu().numpy()[:, m:], 0.5)
+
+
+def test_route_xhc_workload_sampled():
+    """T=8192, N=16, k=4, m=2, C=2048: all tokens routed on the GPU, 64 sampled tokens
+    compared (score gaps > 1e-4 after redrawing)."""
+    inp, _ = xhc_full()
+    rng = np.random.default_rng(3)
+    toks = np.unique(np.concatenate([[0, 8191], rng.choice(8192, 62, replace=False)]))
+    _route_check(inp, toks)
