@@ -90,7 +90,7 @@ __device__ __forceinline__ void sinkhorn_regs(float (&m)[N][N], int iters) {
             float s = 0.0f;
 #pragma unroll
             for (int i = 0; i < N; ++i) s += m[i][j];
-            const float inv = 1.0f / s;
+            const float inv = __frcp_rn(s);      // correctly rounded, = 1.0f / s
 #pragma unroll
             for (int i = 0; i < N; ++i) m[i][j] *= inv;
         }
@@ -99,49 +99,10 @@ __device__ __forceinline__ void sinkhorn_regs(float (&m)[N][N], int iters) {
             float s = 0.0f;
 #pragma unroll
             for (int j = 0; j < N; ++j) s += m[i][j];
-            const float inv = 1.0f / s;
+            const float inv = __frcp_rn(s);
 #pragma unroll
             for (int j = 0; j < N; ++j) m[i][j] *= inv;
         }
-    }
-}
-
-// Row-parallel Sinkhorn-Knopp over an aligned group of 8 lanes (N <= 8):
-// lane g < N of the group holds row g of the logits in `row`; lanes g >= N
-// hold anything and end with zeros.  Same arithmetic as sinkhorn_regs (per
-// column maximum shift when iters >= 1, then `iters` x {columns, rows}); the
-// column sums are butterfly reductions over the 8 lanes.  Every lane of the
-// warp must call it (it shuffles over the full warp).
-template <int N>
-__device__ __forceinline__ void sinkhorn_group8(float (&row)[N], int g, int iters) {
-    const bool live = g < N;
-#pragma unroll
-    for (int j = 0; j < N; ++j) {
-        float mx = live ? row[j] : -INFINITY;
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-        if (iters == 0) mx = 0.0f;
-        row[j] = live ? expf(row[j] - mx) : 0.0f;
-    }
-    for (int it = 0; it < iters; ++it) {
-        float cs[N];
-#pragma unroll
-        for (int j = 0; j < N; ++j) {
-            cs[j] = row[j];
-            cs[j] += __shfl_xor_sync(0xffffffffu, cs[j], 1);
-            cs[j] += __shfl_xor_sync(0xffffffffu, cs[j], 2);
-            cs[j] += __shfl_xor_sync(0xffffffffu, cs[j], 4);
-        }
-        float rs = 0.0f;
-#pragma unroll
-        for (int j = 0; j < N; ++j) {
-            row[j] *= 1.0f / cs[j];
-            rs += row[j];
-        }
-        const float inv = live ? 1.0f / rs : 0.0f;
-#pragma unroll
-        for (int j = 0; j < N; ++j) row[j] *= inv;
     }
 }
 

@@ -13,19 +13,19 @@
 //          it runs at most LAG tiles ahead of the x_in warps, which keeps the
 //          x_in re-read inside L2.
 //   1      MMA issuer: D[128 x NB] += X_chunk[128 x 64] * phiT_chunk[NB x 64]^T
-//          (tcgen05.mma kind::f16, fp32 accumulator in TMEM, double-buffered
-//          across tiles; rows >= Mt are never read).
-//   2-3    sum of squares of every tile row of every ring stage (Eq.15),
-//          handed to the epilogue through a double-buffered shared array.
+//          and S[128 x 64] += X_chunk * X_chunk[0..63]^T, whose diagonal is
+//          each row's sum of squares (Eq.15) (tcgen05.mma kind::f16, fp32
+//          accumulators in TMEM, double-buffered across tiles; rows >= Mt are
+//          never read).  The MMA commit is the only consumer of a ring stage.
 //   4-5    epilogue: each tile row's partial (logits, sum of squares) from TMEM
 //          is pushed with st.async into the shared memory of the CTA that owns
 //          the token (8 tokens per CTA); the owner reduces the 8 partial rows,
-//          computes the coefficients (Eq.16-19; row-parallel Sinkhorn over 8
-//          lanes) and pushes H_pre to every CTA of the cluster.  The pushes
+//          computes the coefficients (Eq.16-19, Sinkhorn in registers) and
+//          pushes H_pre to every CTA of the cluster.  The pushes
 //          complete transactions on the receivers' mbarriers, so no fence or
 //          remote arrive sits on this path.
-//   6-15   x_in = H_pre X for this CTA's channels, re-reading the tile's X
-//          slice from L2 (evict-first on this last read).
+//   2-3, 6-15  x_in = H_pre X for this CTA's channels, re-reading the tile's
+//          X slice from L2 (evict-first on this last read).
 // The roles meet only through mbarriers and one progress counter, so the TMA
 // ring keeps streaming while a tile's coefficients and x_in are produced.
 //
@@ -49,9 +49,8 @@ constexpr int KC = 64;           // K elements per chunk (one 128-byte row)
 constexpr int STAGE_BYTES = MT_CAP * 128;
 constexpr int STAGES = 14;
 constexpr int NTHREADS = 512;
-constexpr int SS_WARP0 = 2, SS_WARPS = 2;                  // one tile row per thread
-constexpr int EPI_WARP0 = 4, EPI_WARPS = 2, EPI_THREADS = 64;
-constexpr int XIN_WARP0 = 6, XIN_WARPS = 10, XIN_THREADS = 320;
+constexpr int EPI_WARP0 = 4, EPI_WARPS = 2, EPI_THREADS = 64;   // TMEM lane quarters 0 and 1
+constexpr int XIN_WARPS = 12, XIN_THREADS = 384;                 // warps 2-3 and 6-15
 constexpr int TOK_PER_CTA = MT_CAP / CL;  // tokens whose coefficients a CTA computes
 constexpr int XIN_UNROLL = 4;             // x_in vectors in flight per thread
 constexpr int LAG = 2;                    // tiles the TMA stream may run ahead of x_in
@@ -63,15 +62,15 @@ template <int N> struct Cfg {
     static constexpr int NB = (P + 15) / 16 * 16;  // MMA N
     static constexpr int PS = P + 1;               // partial row: P logits + sum of squares
     static constexpr int PSP = (PS + 3) / 4 * 4;   // ... padded to 16-byte multiples
-    static constexpr int TMEM_COLS = (2 * NB <= 32) ? 32 : (2 * NB <= 64 ? 64 : (2 * NB <= 128 ? 128 : 256));
+    static constexpr int SQ_COL = 2 * NB;           // X X^T accumulators (2 x MT_CAP columns) after the logits
+    static constexpr int TMEM_COLS = 256;
 };
 
 enum Bar { B_FULL = 0, B_EMPTY = B_FULL + STAGES, B_TFULL = B_EMPTY + STAGES, B_TEMPTY = B_TFULL + 2,
-           B_SSFULL = B_TEMPTY + 2, B_SSEMPTY = B_SSFULL + 2, B_PART = B_SSEMPTY + 2, B_HPRE,
-           B_XIN = B_HPRE + 2, B_PHI, B_DRAIN, B_COUNT };
+           B_PART = B_TEMPTY + 2, B_HPRE, B_XIN = B_HPRE + 2, B_PHI, B_DRAIN, B_COUNT };
 
 struct Layout {
-    uint32_t phi, ring, part, ss, hpre, bars, slot, total;
+    uint32_t phi, ring, part, hpre, bias, bars, slot, total;
 };
 
 template <int N>
@@ -81,9 +80,9 @@ __host__ __device__ inline Layout layout_for(int NQ) {
     L.phi = 0;
     L.ring = uint32_t(NQ) * G::R * 128;                      // multiple of 1024
     L.part = L.ring + STAGES * STAGE_BYTES;
-    L.ss = L.part + CL * TOK_PER_CTA * G::PSP * 4;         // [source CTA][token][PSP]
-    L.hpre = L.ss + 2 * MT_CAP * 4;
-    L.bars = (L.hpre + 2 * MT_CAP * N * 4 + 15) / 16 * 16;
+    L.hpre = L.part + CL * TOK_PER_CTA * G::PSP * 4;       // after [source CTA][token][PSP]
+    L.bias = L.hpre + 2 * MT_CAP * N * 4;
+    L.bars = (L.bias + G::P * 4 + 15) / 16 * 16;
     L.slot = L.bars + B_COUNT * 8;
     L.total = L.slot + 16;
     // The MMA reads 128 rows from a stage's base: the last stage's rows past
@@ -115,15 +114,13 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     uint8_t* sphi = smem + L.phi;
     uint8_t* sring = smem + L.ring;
     float* rpart = reinterpret_cast<float*>(smem + L.part);   // [CL][TOK_PER_CTA][PSP], pushed by the cluster
-    float* sss = reinterpret_cast<float*>(smem + L.ss);       // [2][MT_CAP]
     float* shpre = reinterpret_cast<float*>(smem + L.hpre);   // [2][MT_CAP][N]
+    float* sb = reinterpret_cast<float*>(smem + L.bias);      // b, kept on chip for the coefficients
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
     uint64_t* full = bars + B_FULL;
     uint64_t* empty = bars + B_EMPTY;
     uint64_t* tfull = bars + B_TFULL;
     uint64_t* tempty = bars + B_TEMPTY;
-    uint64_t* ssfull = bars + B_SSFULL;
-    uint64_t* ssempty = bars + B_SSEMPTY;
     uint64_t* part_full = bars + B_PART;     // this CTA's tokens: all CL partial rows landed
     uint64_t* hpre_full = bars + B_HPRE;     // [2] H_pre of every tile row landed (per tile parity)
     uint64_t* xin_prog = bars + B_XIN;
@@ -144,13 +141,11 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         s_xin_done = 0;
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1 + SS_WARPS);
+            mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
             mbar_init(&tempty[a], EPI_WARPS);
-            mbar_init(&ssfull[a], SS_WARPS);
-            mbar_init(&ssempty[a], EPI_WARPS);
         }
         // one local arrival (with the expected byte count) per phase; the bytes
         // come from st.async pushes of the cluster
@@ -163,6 +158,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(slot, G::TMEM_COLS);
+    for (int p = threadIdx.x; p < P; p += NTHREADS) sb[p] = b[p];
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *slot;
@@ -221,6 +217,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(MROWS, NB);
+            constexpr uint32_t idesc_sq = idesc_bf16_f32(MROWS, MT_CAP);   // X X^T, tile rows only
             const uint32_t ring_a = smem_u32(sring), phi_a = smem_u32(sphi);
             int s = 0, it = 0;
             uint32_t ph = 0;
@@ -230,6 +227,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 if (!mbar_wait(&tempty[acc], (uint32_t((it >> 1) & 1)) ^ 1)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d = tmem_base + uint32_t(acc * NB);
+                const uint32_t dsq = tmem_base + uint32_t(G::SQ_COL + acc * MT_CAP);
                 for (int q = 0; q < NQ; ++q) {
                     if (!mbar_wait(&full[s], ph) || *(volatile int*)&s_abort) { ok = false; break; }
                     tc_fence_after();
@@ -238,6 +236,8 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                         const uint64_t ad = sdesc_k_sw128(ring_a + s * STAGE_BYTES + kk * 32);
                         const uint64_t bd = sdesc_k_sw128(phi_a + q * R * 128 + kk * 32);
                         mma_bf16(d, ad, bd, idesc, (q | kk) != 0);
+                        // Eq.(15): the sums of squares are the diagonal of X X^T (B = the same rows)
+                        mma_bf16(dsq, ad, ad, idesc_sq, (q | kk) != 0);
                     }
                     mma_commit(&empty[s]);
                     if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -250,40 +250,8 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 mbar_wait(drain, 0, 1ll << 22);
             }
         }
-    } else if (warp < EPI_WARP0) {
-        // ------------------------------------------------------------ sum of squares
-        const int r0 = (warp - SS_WARP0) * 32 + lane;   // tile row of this thread
-        int s = 0, it = 0;
-        uint32_t ph = 0;
-        for (int tile = cluster_id; tile < num_tiles; tile += nclusters, ++it) {
-            const int acc = it & 1;
-            bool ok = mbar_wait(&ssempty[acc], (uint32_t((it >> 1) & 1)) ^ 1);
-            float ssa = 0.0f, ssb = 0.0f;
-            for (int q = 0; q < NQ && ok; ++q) {
-                if (!mbar_wait(&full[s], ph) || *(volatile int*)&s_abort) { ok = false; break; }
-                const uint4* ra = reinterpret_cast<const uint4*>(sring + s * STAGE_BYTES + r0 * 128);
-#pragma unroll
-                for (int g = 0; g < 8; g += 2) {
-                    const uint4 va = ra[g], vb = ra[g + 1];
-                    const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        float x0 = bf16_lo(wa[h]), x1 = bf16_hi(wa[h]);
-                        ssa = fmaf(x0, x0, ssa); ssa = fmaf(x1, x1, ssa);
-                        x0 = bf16_lo(wb[h]); x1 = bf16_hi(wb[h]);
-                        ssb = fmaf(x0, x0, ssb); ssb = fmaf(x1, x1, ssb);
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
-                if (++s == STAGES) { s = 0; ph ^= 1; }
-            }
-            if (!ok) { s_abort = 1; break; }
-            sss[acc * MT_CAP + r0] = ssa + ssb;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&ssfull[acc]);
-        }
-    } else if (warp < XIN_WARP0) {
+
+    } else if (warp == EPI_WARP0 || warp == EPI_WARP0 + 1) {
         // ------------------------------------------------------------ epilogue
         const int et = threadIdx.x - EPI_WARP0 * 32;    // 0..63
         const int qd = warp & 3;                        // TMEM lane quarter of this warp (0, 1)
@@ -305,7 +273,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 mbar_arrive_expect_tx(part_full, PART_BYTES);
                 mbar_arrive_expect_tx(&hpre_full[acc], HPRE_BYTES);
             }
-            if (!mbar_wait(&tfull[acc], par) || !mbar_wait(&ssfull[acc], par)) { s_abort = 1; break; }
+            if (!mbar_wait(&tfull[acc], par)) { s_abort = 1; break; }
             tc_fence_after();
             float d[NB];
             const uint32_t taddr = tmem_base + (uint32_t(qd * 32) << 16) + uint32_t(acc * NB);
@@ -317,10 +285,22 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
 #pragma unroll
                 for (int j = 0; j < 16; ++j) d[c + j] = tmp[j];
             }
-            const float ss = sss[acc * MT_CAP + m];
+            float ss = 0.0f;
+            {
+                const uint32_t qaddr = tmem_base + (uint32_t(qd * 32) << 16) +
+                                       uint32_t(G::SQ_COL + acc * MT_CAP + qd * 32);
+#pragma unroll
+                for (int c = 0; c < 32; c += 16) {
+                    float tmp[16];
+                    tmem_ld16(qaddr + c, tmp);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) if (c + j == lane) ss = tmp[j];   // diagonal (m, m)
+                }
+            }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) { mbar_arrive(&tempty[acc]); mbar_arrive(&ssempty[acc]); }
+            if (lane == 0) mbar_arrive(&tempty[acc]);
 
             // H_pre of tile it lands in buffer it&1, last read by the x_in warps for
             // tile it-2: they must have moved on (they arrive after their tile it-1 wait)
@@ -358,19 +338,26 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 }
                 const float r = sqrtf(v[P] * inv_K + eps);                     // Eq.(15)
                 const float inv_r = 1.0f / r;
+                // every lane of the group carries the whole n x n Sinkhorn (no shuffles in
+                // the iterations); lane g < N then keeps stream g's gates and H_res row g
+                float mres[N][N];
+#pragma unroll
+                for (int i = 0; i < N; ++i)
+#pragma unroll
+                    for (int k = 0; k < N; ++k)
+                        mres[i][k] = a2 * v[2 * N + i * N + k] * inv_r + sb[2 * N + i * N + k];   // Eq.(16)
+                sinkhorn_regs<N>(mres, t_iters);                                   // Eq.(19)
                 float zpre = 0.0f, zpost = 0.0f, row[N];
 #pragma unroll
                 for (int k = 0; k < N; ++k) row[k] = 0.0f;
 #pragma unroll
                 for (int i = 0; i < N; ++i)
                     if (g == i) {
-                        zpre = a0 * v[i] * inv_r + __ldg(b + i);                   // Eq.(16)
-                        zpost = a1 * v[N + i] * inv_r + __ldg(b + N + i);
+                        zpre = a0 * v[i] * inv_r + sb[i];
+                        zpost = a1 * v[N + i] * inv_r + sb[N + i];
 #pragma unroll
-                        for (int k = 0; k < N; ++k)
-                            row[k] = a2 * v[2 * N + i * N + k] * inv_r + __ldg(b + 2 * N + i * N + k);
+                        for (int k = 0; k < N; ++k) row[k] = mres[i][k];
                     }
-                sinkhorn_group8<N>(row, g, t_iters);                               // Eq.(19)
                 if (g < N) {
                     const float hp = sigmoidf_(zpre);                              // Eq.(17)
                     // every CTA needs H_pre of every tile row for its x_in channels
@@ -392,12 +379,12 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         }
     } else {
         // ------------------------------------------------------------ x_in
-        const int xt = threadIdx.x - XIN_WARP0 * 32;    // 0..XIN_THREADS-1
+        const int xt = (warp < EPI_WARP0 ? warp - 2 : warp - 4) * 32 + lane;   // 0..XIN_THREADS-1
         const uint64_t drop = policy_evict_first();
         const int VPT = Cs / 8;                          // 16-byte vectors per token
         int it = 0;
         for (int tile = cluster_id; tile < num_tiles; tile += nclusters, ++it) {
-            if (!mbar_wait(&hpre_full[it & 1], uint32_t((it >> 1) & 1))) { s_abort = 1; break; }
+            if (!mbar_wait_sleep(&hpre_full[it & 1], uint32_t((it >> 1) & 1))) { s_abort = 1; break; }
             __syncwarp();
             if (lane == 0) mbar_arrive(xin_prog);
             const int64_t t0 = int64_t(tile) * Mt;

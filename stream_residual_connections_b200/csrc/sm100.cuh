@@ -106,6 +106,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
     return false;
 }
 
+// Bounded wait for warps off the critical path: backs off with __nanosleep so
+// that spinning does not take issue slots from the warps it waits for.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
+    const long long cap = g_wait_limit;
+    unsigned ns = 32;
+    for (long long i = 0; i < cap; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        __nanosleep(ns);
+        if (ns < 512) ns <<= 1;
+    }
+    atomicOr(&g_device_error, 1u);
+    return false;
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -87,13 +87,18 @@ route_kernel(const TX* __restrict__ X, const TX* __restrict__ phiT, float a_pre,
     if (stream && Hpre) Hpre[t * N + lane] = hp;
     if (routed && score) score[t * (N - m) + lane - m] = sc;
 
-    // dense read: x_in = sum_i H_pre[i] X[i]
+    // dense read: x_in = sum_i H_pre[i] X[i]  (gates gathered while the whole warp is converged)
+    float hall[NMAX];
+#pragma unroll
+    for (int i = 0; i < NMAX; ++i) hall[i] = __shfl_sync(0xffffffffu, hp, i);
     for (int c0 = lane * W; c0 < C; c0 += 32 * W) {
         float o[W];
 #pragma unroll
         for (int e = 0; e < W; ++e) o[e] = 0.0f;
-        for (int i = 0; i < N; ++i) {
-            const float h = __shfl_sync(0xffffffffu, hp, i);
+#pragma unroll
+        for (int i = 0; i < NMAX; ++i) {
+            if (i >= N) break;
+            const float h = hall[i];
             float xv[W];
             load16<false>(x + int64_t(i) * C + c0, xv);
 #pragma unroll
