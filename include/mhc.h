@@ -177,6 +177,33 @@ mhc_status xhc_sparse_update(void* X, mhc_dtype dt, const float* V, int Kr, cons
                              const float* b_act, int64_t T, int N, int C, int k, int t_iters,
                              float eps, float* H_res, float* H_post, void* stream);
 
+/*
+ * mhc_backward -- gradients of one mHC sublayer (mhc_pre + mhc_post) with all
+ * t_iters Sinkhorn-Knopp iterations unrolled.  [mHC] section 4.3.1 (the
+ * backward of the projection and of the Sinkhorn kernel, which recomputes
+ * the intermediates on chip).  The forward is recomputed from X; nothing from
+ * a forward call is needed.
+ *
+ * Given upstream gradients dX_next (of X_next) and dx_in (of x_in):
+ *   dX     [T][n][C], dtype dt    dL/dX (through x_in, X_next and the coefficients)
+ *   dF_out [T][C],    dtype dt    dL/dF_out = sum_i H_post[i] dX_next[i]
+ *   dphi   [P][n*C]   fp32        dL/dphi in phi's (transposed) layout, summed over tokens
+ *   dalpha [3] fp32 (device), db [P] fp32 (device): summed over tokens
+ * All three sums are overwritten, not accumulated; their summation order is
+ * fixed, so results are bitwise reproducible.  Inputs: as mhc_pre/mhc_post
+ * (phi [P][n*C] transposed, dtype dt; alpha HOST float[3]; b [P] fp32).
+ *   workspace: device scratch of at least mhc_backward_workspace_bytes(T, n, C)
+ *   bytes, 256-byte aligned, owned by the caller; its contents on entry are
+ *   ignored and on exit undefined.
+ * This build: n <= 4, C % 64 == 0, t_iters <= 100.  T == 0 zeroes the sums.
+ */
+size_t mhc_backward_workspace_bytes(int64_t T, int n, int C);
+mhc_status mhc_backward(const void* X, const void* F_out, const void* phi, mhc_dtype dt,
+                        const float* alpha, const float* b, const void* dX_next, const void* dx_in,
+                        int64_t T, int n, int C, int t_iters, float eps, void* dX, void* dF_out,
+                        float* dphi, float* dalpha, float* db, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
 /* Kernel selection for the projection of mhc_pre. */
 typedef enum {
     MHC_PATH_AUTO = 0,    /* tensor cores where supported, else CUDA cores (default) */

@@ -34,6 +34,9 @@
  */
 #include <math.h>
 #include <stdint.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 #include <stdlib.h>
 #include <string.h>
 
@@ -165,7 +168,22 @@ void orc_mhc_backward(const double* X, const double* F, const double* phi,
     memset(dphi, 0, sizeof(double) * K * P);
     memset(dalpha, 0, sizeof(double) * 3);
     memset(db, 0, sizeof(double) * P);
-    for (int64_t t = 0; t < T; ++t) {
+    /* Tokens are split into fixed contiguous ranges, one per thread; each range
+     * sums into its own partial dphi/dalpha/db, and the partials are added in
+     * range order, so the result does not depend on scheduling. */
+    int nthr = 1;
+#ifdef _OPENMP
+    nthr = omp_get_max_threads();
+#endif
+    if (nthr > T) nthr = T > 0 ? (int)T : 1;
+    double* part = (double*)calloc((size_t)nthr * (K * P + 3 + P), sizeof(double));
+#pragma omp parallel for schedule(static, 1) num_threads(nthr)
+    for (int th = 0; th < nthr; ++th) {
+    double* pphi = part + (size_t)th * (K * P + 3 + P);
+    double* palpha = pphi + K * P;
+    double* pdb = palpha + 3;
+    const int64_t t_lo = T * th / nthr, t_hi = T * (th + 1) / nthr;
+    for (int64_t t = t_lo; t < t_hi; ++t) {
         const double* x = X + t * K;
         const double* f = F + t * C;
         const double* gn = dXn + t * K;
@@ -248,8 +266,8 @@ void orc_mhc_backward(const double* X, const double* F, const double* phi,
         double dr = 0.0, dd[8 * 8 + 16];
         for (int p = 0; p < P; ++p) {
             const int s = p < n ? 0 : (p < 2 * n ? 1 : 2);
-            dalpha[s] += dz[p] * d[p] / r;
-            db[p] += dz[p];
+            palpha[s] += dz[p] * d[p] / r;
+            pdb[p] += dz[p];
             dd[p] = aseg[p] * dz[p] / r;
             dr -= aseg[p] * dz[p] * d[p] / (r * r);
         }
@@ -257,11 +275,19 @@ void orc_mhc_backward(const double* X, const double* F, const double* phi,
             double a = 0.0;
             for (int p = 0; p < P; ++p) {
                 a += phi[k * P + p] * dd[p];
-                dphi[k * P + p] += x[k] * dd[p];
+                pphi[k * P + p] += x[k] * dd[p];
             }
             gx[k] += a + dr * x[k] / ((double)K * r);
         }
     }
+    }
+    for (int th = 0; th < nthr; ++th) {
+        const double* pphi = part + (size_t)th * (K * P + 3 + P);
+        for (int64_t e = 0; e < K * P; ++e) dphi[e] += pphi[e];
+        for (int s = 0; s < 3; ++s) dalpha[s] += pphi[K * P + s];
+        for (int p = 0; p < P; ++p) db[p] += pphi[K * P + 3 + p];
+    }
+    free(part);
 }
 
 /* ---------------------------------------------------------------- xHC */

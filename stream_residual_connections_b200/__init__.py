@@ -47,12 +47,16 @@ def _load():
     L.mhc_sync_status.argtypes = [vp]
     L.mhc_set_path.argtypes = [i32]
     L.xhc_route.argtypes = [vp, i32, vp, fp, vp, i64, i32, i32, i32, i32, f32, vp, vp, vp, vp, vp, vp]
+    L.mhc_backward_workspace_bytes.argtypes = [i64, i32, i32]
+    L.mhc_backward_workspace_bytes.restype = ct.c_size_t
+    L.mhc_backward.argtypes = [vp, vp, vp, i32, fp, vp, vp, vp, i64, i32, i32, i32, f32, vp, vp, vp, vp,
+                               vp, vp, ct.c_size_t, vp]
     L.xhc_conv_gs.argtypes = [vp, i32, vp, ct.POINTER(ct.c_int), i32, i64, i32, i64, vp, vp]
     L.xhc_sparse_update.argtypes = [vp, i32, vp, i32, vp, vp, vp, fp, vp, i64, i32, i32, i32, i32,
                                     f32, vp, vp, vp]
     L.mhc_set_wait_limit.argtypes = [ct.c_longlong]
     for name in ("mhc_pre", "mhc_post", "mhc_sync_status", "mhc_set_path", "mhc_set_wait_limit",
-                 "xhc_conv_gs", "xhc_sparse_update", "xhc_route"):
+                 "xhc_conv_gs", "xhc_sparse_update", "xhc_route", "mhc_backward"):
         getattr(L, name).restype = ct.c_int
     return L
 
@@ -210,3 +214,29 @@ def xhc_route(X, phi_read, alpha_read, b_read, k: int, m: int, eps: float = 1e-6
                               C, int(k), int(m), float(eps), _ptr(x_in), _ptr(H_pre), _ptr(score),
                               _ptr(idx), _ptr(w), _stream(stream)))
     return x_in, H_pre, score, idx, w
+
+
+def mhc_backward_workspace_bytes(T: int, n: int, C: int) -> int:
+    return int(native().mhc_backward_workspace_bytes(int(T), int(n), int(C)))
+
+
+def mhc_backward(X, F_out, phi, alpha, b, dX_next, dx_in, t_iters: int = 20, eps: float = 1e-6, *,
+                 dX=None, dF=None, dphi=None, dalpha=None, db=None, workspace=None, stream=None):
+    """Gradients of one mHC sublayer (see include/mhc.h).  phi is [P][nC] (transposed).
+    Returns (dX, dF, dphi [P][nC] fp32, dalpha [3], db [P])."""
+    T, n, C = X.shape
+    P = n * n + 2 * n
+    dev = X.device
+    dX = torch.empty_like(X) if dX is None else dX
+    dF = torch.empty_like(F_out) if dF is None else dF
+    dphi = torch.empty((P, n * C), dtype=torch.float32, device=dev) if dphi is None else dphi
+    dalpha = torch.empty(3, dtype=torch.float32, device=dev) if dalpha is None else dalpha
+    db = torch.empty(P, dtype=torch.float32, device=dev) if db is None else db
+    need = mhc_backward_workspace_bytes(T, n, C)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(native().mhc_backward(_ptr(X), _ptr(F_out), _ptr(phi), _dt(X), _host3(alpha), _ptr(b),
+                                 _ptr(dX_next), _ptr(dx_in), T, n, C, int(t_iters), float(eps), _ptr(dX),
+                                 _ptr(dF), _ptr(dphi), _ptr(dalpha), _ptr(db), ct.c_void_p(workspace.data_ptr()),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)))
+    return dX, dF, dphi, dalpha, db

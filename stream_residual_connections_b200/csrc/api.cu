@@ -257,6 +257,76 @@ mhc_status xhc_sparse_update(void* X, mhc_dtype dt, const float* V, int Kr, cons
     return launch_sparse_update(a, static_cast<cudaStream_t>(stream));
 }
 
+size_t mhc_backward_workspace_bytes(int64_t T, int n, int C)
+{
+    (void)C;
+    const size_t stride = backward_record_stride(n);
+    if (T < 0 || stride == 0) return 0;
+    const size_t P = size_t(n) * n + 2 * n;
+    const size_t floats = size_t(T) * stride + size_t(T) * P + size_t(T);
+    return ((floats * 4 + 255) / 256) * 256 + 256;
+}
+
+mhc_status mhc_backward(const void* X, const void* F_out, const void* phi, mhc_dtype dt, const float* alpha,
+                        const float* b, const void* dX_next, const void* dx_in, int64_t T, int n, int C,
+                        int t_iters, float eps, void* dX, void* dF_out, float* dphi, float* dalpha,
+                        float* db, void* workspace, size_t workspace_bytes, void* stream)
+{
+    const char* fn = "mhc_backward";
+    g_msg[0] = 0;
+    REQUIRE(valid_dt(dt), MHC_ERR_INVALID_ARG, "%s: unknown dtype", fn);
+    REQUIRE(n >= 1 && n <= 8, MHC_ERR_INVALID_ARG, "%s: n=%d outside [1, 8]", fn, n);
+    REQUIRE(C > 0 && C % 8 == 0, MHC_ERR_INVALID_ARG, "%s: C=%d must be a positive multiple of 8", fn, C);
+    REQUIRE(T >= 0, MHC_ERR_INVALID_ARG, "%s: T=%lld < 0", fn, (long long)T);
+    REQUIRE(t_iters >= 0 && t_iters <= 1000, MHC_ERR_INVALID_ARG, "%s: t_iters=%d outside [0, 1000]", fn, t_iters);
+    REQUIRE(eps >= 0.0f, MHC_ERR_INVALID_ARG, "%s: eps < 0", fn);
+    REQUIRE(alpha != nullptr, MHC_ERR_INVALID_ARG, "%s: alpha (host float[3]) is NULL", fn);
+    REQUIRE(n <= 4 && C % 64 == 0 && t_iters <= 100, MHC_ERR_UNSUPPORTED,
+            "%s: this build needs n <= 4, C %% 64 == 0, t_iters <= 100", fn);
+    const int P = n * n + 2 * n;
+    REQUIRE_PTR(dphi, "dphi");
+    REQUIRE(dalpha != nullptr && db != nullptr, MHC_ERR_INVALID_ARG, "%s: dalpha or db is NULL", fn);
+    if (T == 0) {
+        // empty batch: every gradient sum is zero
+        cudaStream_t s = static_cast<cudaStream_t>(stream);
+        mhc_status st = cuda_status(cudaMemsetAsync(dphi, 0, size_t(P) * n * C * 4, s), fn);
+        if (st == MHC_OK) st = cuda_status(cudaMemsetAsync(dalpha, 0, 3 * 4, s), fn);
+        if (st == MHC_OK) st = cuda_status(cudaMemsetAsync(db, 0, size_t(P) * 4, s), fn);
+        return st;
+    }
+    REQUIRE_PTR(X, "X");
+    REQUIRE_PTR(F_out, "F_out");
+    REQUIRE_PTR(phi, "phi");
+    REQUIRE(b != nullptr, MHC_ERR_INVALID_ARG, "%s: b is NULL", fn);
+    REQUIRE_PTR(dX_next, "dX_next");
+    REQUIRE_PTR(dx_in, "dx_in");
+    REQUIRE_PTR(dX, "dX");
+    REQUIRE_PTR(dF_out, "dF_out");
+    REQUIRE(workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 255u) == 0, MHC_ERR_INVALID_ARG,
+            "%s: workspace must be non-NULL and 256-byte aligned", fn);
+    const size_t need = mhc_backward_workspace_bytes(T, n, C);
+    REQUIRE(workspace_bytes >= need, MHC_ERR_INVALID_ARG, "%s: workspace of %zu bytes < %zu needed", fn,
+            workspace_bytes, need);
+    const size_t es = dt_size(dt);
+    const Range ins[8] = {range_of(X, size_t(T) * n * C * es), range_of(F_out, size_t(T) * C * es),
+                          range_of(phi, size_t(P) * n * C * es), range_of(b, size_t(P) * 4),
+                          range_of(dX_next, size_t(T) * n * C * es), range_of(dx_in, size_t(T) * C * es),
+                          range_of(workspace, need), range_of(alpha, 0)};
+    const Range outs[5] = {range_of(dX, size_t(T) * n * C * es), range_of(dF_out, size_t(T) * C * es),
+                           range_of(dphi, size_t(P) * n * C * 4), range_of(dalpha, 12), range_of(db, size_t(P) * 4)};
+    for (int o = 0; o < 5; ++o) {
+        for (int i = 0; i < 7; ++i)
+            REQUIRE(!overlap(outs[o], ins[i]), MHC_ERR_INVALID_ARG, "%s: an output overlaps an input or the workspace", fn);
+        for (int q = 0; q < o; ++q)
+            REQUIRE(!overlap(outs[o], outs[q]), MHC_ERR_INVALID_ARG, "%s: outputs overlap", fn);
+    }
+    float* ws = static_cast<float*>(workspace);
+    const size_t stride = backward_record_stride(n);
+    BwdArgs a{X, F_out, phi, dt, {alpha[0], alpha[1], alpha[2]}, b, dX_next, dx_in, T, n, C, t_iters, eps,
+              dX, dF_out, dphi, dalpha, db, ws, ws + size_t(T) * stride, ws + size_t(T) * stride + size_t(T) * P};
+    return launch_backward(a, static_cast<cudaStream_t>(stream));
+}
+
 mhc_status mhc_set_path(mhc_path path)
 {
     g_msg[0] = 0;

@@ -18,6 +18,9 @@ struct PreArgs {
     const float* b;
     int64_t T; int n; int C; int t_iters; float eps;
     void* x_in; float* H_pre; float* H_post; float* H_res;
+    // internal (the backward's recompute): u = (x phi)/r [T][P] and r [T] when
+    // non-null; skip_xin leaves x_in unwritten; H_post / H_res may then be null
+    float* u_out = nullptr; float* r_out = nullptr; bool skip_xin = false;
 };
 
 // CUDA-core (FMA) projection path: every n, dtype pair and C % 8 == 0.
@@ -45,6 +48,15 @@ struct RouteArgs {
     void* x_in; float* H_pre; float* score; int32_t* idx; float* w;
 };
 mhc_status launch_route(const RouteArgs& a, cudaStream_t s);
+
+struct BwdArgs {
+    const void* X; const void* F; const void* phi; mhc_dtype dt; float alpha[3]; const float* b;
+    const void* dXn; const void* dxin; int64_t T; int n; int C; int t_iters; float eps;
+    void* dX; void* dF; float* dphi; float* dalpha; float* db;
+    float* records; float* u_scratch; float* r_scratch;   // carved from the caller's workspace
+};
+size_t backward_record_stride(int n);            // floats per token record (0: unsupported n)
+mhc_status launch_backward(const BwdArgs& a, cudaStream_t s);
 
 // Which mhc_pre path to take (MHC_PRE_PATH_*), process-wide.
 extern int g_pre_path;

@@ -7,3 +7,4 @@
 #include "xhc_conv_gs.cu"
 #include "xhc_update.cu"
 #include "xhc_route.cu"
+#include "mhc_bwd.cu"

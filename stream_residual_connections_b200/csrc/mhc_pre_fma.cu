@@ -27,7 +27,7 @@ __global__ void __launch_bounds__(256)
 pre_fma_kernel(const TX* __restrict__ X, const TP* __restrict__ phiT, float a0, float a1, float a2,
                const float* __restrict__ b, int64_t T, int C, int t_iters, float eps,
                TX* __restrict__ x_in, float* __restrict__ Hpre, float* __restrict__ Hpost,
-               float* __restrict__ Hres)
+               float* __restrict__ Hres, float* __restrict__ u_out, float* __restrict__ r_out)
 {
     constexpr int P = N * N + 2 * N;
     constexpr int W = Vec<TX>::W;            // X elements per 16-byte load
@@ -83,11 +83,17 @@ pre_fma_kernel(const TX* __restrict__ X, const TP* __restrict__ phiT, float a0, 
 #pragma unroll
         for (int i = 0; i < N; ++i) {
             if (Hpre) Hpre[t * N + i] = hpre[i];
-            Hpost[t * N + i] = hpost[i];
+            if (Hpost) Hpost[t * N + i] = hpost[i];
 #pragma unroll
-            for (int j = 0; j < N; ++j) Hres[(t * N + i) * N + j] = m[i][j];
+            for (int j = 0; j < N; ++j) if (Hres) Hres[(t * N + i) * N + j] = m[i][j];
+        }
+        if (u_out) {
+#pragma unroll
+            for (int p = 0; p < P; ++p) u_out[t * P + p] = acc[p] * inv_r;
+            r_out[t] = r;
         }
     }
+    if (!x_in) return;
 
     // F_pre: x_in = sum_i H_pre[i] X[i].
     for (int c0 = lane * W; c0 < C; c0 += 32 * W) {
@@ -112,8 +118,8 @@ static mhc_status launch_pre_fma_n(const PreArgs& a, cudaStream_t s)
     const int64_t blocks = (a.T + warps - 1) / warps;
     pre_fma_kernel<N, TX, TP><<<dim3(unsigned(blocks)), warps * 32, 0, s>>>(
         static_cast<const TX*>(a.X), static_cast<const TP*>(a.phi), a.alpha[0], a.alpha[1],
-        a.alpha[2], a.b, a.T, a.C, a.t_iters, a.eps, static_cast<TX*>(a.x_in), a.H_pre,
-        a.H_post, a.H_res);
+        a.alpha[2], a.b, a.T, a.C, a.t_iters, a.eps, a.skip_xin ? nullptr : static_cast<TX*>(a.x_in),
+        a.H_pre, a.H_post, a.H_res, a.u_out, a.r_out);
     return launch_status("mhc_pre (fma) kernel");
 }
 

@@ -99,7 +99,8 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
               const bf16_t* __restrict__ X, float a0, float a1, float a2,
               const float* __restrict__ b, int64_t T, int C, int Mt, int num_tiles, int t_iters,
               float eps, bf16_t* __restrict__ x_in, float* __restrict__ Hpre,
-              float* __restrict__ Hpost, float* __restrict__ Hres)
+              float* __restrict__ Hpost, float* __restrict__ Hres, float* __restrict__ u_out,
+              float* __restrict__ r_out)
 {
     using G = Cfg<N>;
     constexpr int P = G::P, R = G::R, NB = G::NB, PS = G::PS, PSP = G::PSP;
@@ -366,11 +367,19 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     for (uint32_t rr = 0; rr < CL; ++rr) st_async_f32(mapa(hoff, rr), hp, mapa(hbar, rr));
                     const int64_t t = t0 + j;
                     if (j < Mt && t < T) {
-                        Hpost[t * N + g] = 2.0f * sigmoidf_(zpost);                // Eq.(18)
+                        if (Hpost) Hpost[t * N + g] = 2.0f * sigmoidf_(zpost);     // Eq.(18)
                         if (Hpre) Hpre[t * N + g] = hp;
+                        if (Hres) {
 #pragma unroll
-                        for (int k = 0; k < N; ++k) Hres[(t * N + g) * N + k] = row[k];
+                            for (int k = 0; k < N; ++k) Hres[(t * N + g) * N + k] = row[k];
+                        }
                     }
+                }
+                if (u_out && j < Mt && t0 + j < T) {       // the backward's recompute
+#pragma unroll
+                    for (int p = 0; p < P; ++p)
+                        if ((p & 7) == g) u_out[(t0 + j) * P + p] = v[p] * inv_r;
+                    if (g == 0) r_out[t0 + j] = r;
                 }
             }
             // every owner has read its partial rows of this tile once this CTA holds the
@@ -390,7 +399,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             const int64_t t0 = int64_t(tile) * Mt;
             const float* hb = shpre + (it & 1) * MT_CAP * N;
             const int rows = int((T - t0) < int64_t(Mt) ? (T - t0) : int64_t(Mt));
-            const int items = rows * VPT;
+            const int items = x_in ? rows * VPT : 0;
             for (int w0 = xt; w0 < items; w0 += XIN_UNROLL * XIN_THREADS) {
                 uint4 raw[XIN_UNROLL][N];
                 int tok[XIN_UNROLL], cc[XIN_UNROLL];
@@ -534,8 +543,8 @@ static mhc_status launch_n(const PreArgs& a, cudaStream_t s)
     }
     kern<<<dim3(unsigned(nclusters * CL)), NTHREADS, size_t(smem), s>>>(
         mapX, mapPhi, static_cast<const bf16_t*>(a.X), a.alpha[0], a.alpha[1], a.alpha[2], a.b, a.T,
-        a.C, Mt, int(tiles64), a.t_iters, a.eps, static_cast<bf16_t*>(a.x_in), a.H_pre, a.H_post,
-        a.H_res);
+        a.C, Mt, int(tiles64), a.t_iters, a.eps, a.skip_xin ? nullptr : static_cast<bf16_t*>(a.x_in),
+        a.H_pre, a.H_post, a.H_res, a.u_out, a.r_out);
     return launch_status("mhc_pre (tc) kernel");
 }
 
