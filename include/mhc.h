@@ -204,6 +204,31 @@ mhc_status mhc_backward(const void* X, const void* F_out, const void* phi, mhc_d
                         float* dphi, float* dalpha, float* db, void* workspace,
                         size_t workspace_bytes, void* stream);
 
+/*
+ * mhc_backward_noalloc -- mhc_backward without a caller workspace.  The pages
+ * have no counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory (code running while a CUDA graph is being captured,
+ * a custom allocator's own callbacks, or an embedding runtime that owns all
+ * allocations and forbids libraries to make any).
+ *
+ * Same arguments, results and restrictions as mhc_backward, minus the
+ * workspace.  The scratch is a fixed MHC_NOALLOC_SCRATCH_BYTES (4 MiB) array
+ * inside the library, held by every GPU that loads the library until the
+ * process exits; batches whose mhc_backward_workspace_bytes(T, n, C) exceeds it
+ * are rejected with MHC_ERR_UNSUPPORTED (at n = 4 that is T > 10,800 or so).
+ * No allocating routine is called.  The first call on each device looks up
+ * the scratch address and should come before any stream capture.  Every call
+ * on a device uses the same scratch: calls whose work overlaps on the GPU
+ * race, so order them (one stream, or events).  Nothing in the scratch needs
+ * to start at zero; it keeps the previous call's leftovers.
+ */
+#define MHC_NOALLOC_SCRATCH_BYTES (4u << 20)
+mhc_status mhc_backward_noalloc(const void* X, const void* F_out, const void* phi, mhc_dtype dt,
+                                const float* alpha, const float* b, const void* dX_next,
+                                const void* dx_in, int64_t T, int n, int C, int t_iters, float eps,
+                                void* dX, void* dF_out, float* dphi, float* dalpha, float* db,
+                                void* stream);
+
 /* Kernel selection for the projection of mhc_pre. */
 typedef enum {
     MHC_PATH_AUTO = 0,    /* tensor cores where supported, else CUDA cores (default) */

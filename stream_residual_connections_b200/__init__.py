@@ -51,12 +51,15 @@ def _load():
     L.mhc_backward_workspace_bytes.restype = ct.c_size_t
     L.mhc_backward.argtypes = [vp, vp, vp, i32, fp, vp, vp, vp, i64, i32, i32, i32, f32, vp, vp, vp, vp,
                                vp, vp, ct.c_size_t, vp]
+    L.mhc_backward_noalloc.argtypes = [vp, vp, vp, i32, fp, vp, vp, vp, i64, i32, i32, i32, f32, vp, vp,
+                                       vp, vp, vp, vp]
     L.xhc_conv_gs.argtypes = [vp, i32, vp, ct.POINTER(ct.c_int), i32, i64, i32, i64, vp, vp]
     L.xhc_sparse_update.argtypes = [vp, i32, vp, i32, vp, vp, vp, fp, vp, i64, i32, i32, i32, i32,
                                     f32, vp, vp, vp]
     L.mhc_set_wait_limit.argtypes = [ct.c_longlong]
     for name in ("mhc_pre", "mhc_post", "mhc_sync_status", "mhc_set_path", "mhc_set_wait_limit",
-                 "xhc_conv_gs", "xhc_sparse_update", "xhc_route", "mhc_backward"):
+                 "xhc_conv_gs", "xhc_sparse_update", "xhc_route", "mhc_backward",
+                 "mhc_backward_noalloc"):
         getattr(L, name).restype = ct.c_int
     return L
 
@@ -239,4 +242,17 @@ def mhc_backward(X, F_out, phi, alpha, b, dX_next, dx_in, t_iters: int = 20, eps
                                  _ptr(dX_next), _ptr(dx_in), T, n, C, int(t_iters), float(eps), _ptr(dX),
                                  _ptr(dF), _ptr(dphi), _ptr(dalpha), _ptr(db), ct.c_void_p(workspace.data_ptr()),
                                  workspace.numel() * workspace.element_size(), _stream(stream)))
+    return dX, dF, dphi, dalpha, db
+
+
+def mhc_backward_noalloc(X, F_out, phi, alpha, b, dX_next, dx_in, t_iters: int = 20, eps: float = 1e-6,
+                         *, dX, dF, dphi, dalpha, db, stream=None):
+    """mhc_backward using the library's built-in scratch instead of a workspace, for
+    callers that cannot allocate (e.g. during CUDA graph capture).  All outputs are
+    caller-provided; see include/mhc.h for the size limit and the sharing rules."""
+    T, n, C = X.shape
+    _check(native().mhc_backward_noalloc(_ptr(X), _ptr(F_out), _ptr(phi), _dt(X), _host3(alpha), _ptr(b),
+                                         _ptr(dX_next), _ptr(dx_in), T, n, C, int(t_iters), float(eps),
+                                         _ptr(dX), _ptr(dF), _ptr(dphi), _ptr(dalpha), _ptr(db),
+                                         _stream(stream)))
     return dX, dF, dphi, dalpha, db

@@ -8,3 +8,4 @@
 #include "xhc_update.cu"
 #include "xhc_route.cu"
 #include "mhc_bwd.cu"
+#include "mhc_bwd_noalloc.cu"
