@@ -45,7 +45,9 @@ FALLBACK_HBM_GBS = 6650.0
 
 
 def algorithmic_bytes(T: int, n: int, C: int, es: int = 2) -> dict:
-    """Bytes each kernel must move per launch (Roofline)."""
+    """Bytes each kernel must move per launch: mhc_pre reads X once, writes x_in and the
+    coefficients, and reads phi once; mhc_post reads X and F_out and the coefficients and
+    writes X_next (the (n+1)C read / nC write count of the fused post kernel)."""
     P = n * n + 2 * n
     pre = T * (n * C * es + C * es + (2 * n + n * n) * 4) + n * C * P * es + P * 4
     post = T * (n * C * es + C * es + (n + n * n) * 4 + n * C * es)

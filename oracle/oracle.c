@@ -19,7 +19,7 @@
  *     (gated projections, Sinkhorn on the active streams, H_post = 2*sigma);
  *     project page "default xHC configuration" table.
  *
- * Readings of points the pages leave open (each listed in the design doc):
+ * Readings of points the pages leave open:
  *   RMSNorm: r = sqrt(sum(x^2)/(nC) + eps), no weight (folded into phi).
  *   vec(X): index i*C + c (streams outer).  phi columns: pre | post | res.
  *   mat(): row-major, H_res[i][j] = z[2n + i*n + j], weighting source stream

@@ -138,7 +138,7 @@ def redraw_rows(X: np.ndarray, rows, seed: int, attempt: int, dtype: str) -> Non
         X[t] = _normal(rng, X.shape[1:], 1.0, dtype)
 
 
-# Named workloads (shapes of the pages' per-sublayer problem).
+# Named workloads: the per-sublayer problem shapes used by the tests and the benchmark.
 WORKLOADS = {
     "mhc_tiny": dict(T=64, n=4, C=256, dtype="f32", seed=0),
     "mhc_llm": dict(T=8192, n=4, C=4096, dtype="bf16", seed=1),

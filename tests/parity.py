@@ -1,6 +1,5 @@
 """Shared helpers of the parity tests: moving the seeded inputs to the device,
-reading results back, and the tolerances (each derived in the design doc,
-"Tolerances").
+reading results back, and the tolerances.
 
 Coefficients (fp32): |gpu - oracle| <= 1e-5 absolute.
 
