@@ -4,35 +4,46 @@
 // [mHC] section 4.3.1, Eq.(14)-(19), and F_pre := H_pre x_l.  Per token tile
 // of Mt <= 64 tokens, the 8 CTAs of a cluster split the C channels: CTA r
 // owns channels [r*C/8, (r+1)*C/8) of every stream, i.e. a K-slice of
-// n*C/8 elements of each token's n*C row, and phi's matching K-slice stays
-// resident in its shared memory for the whole (persistent) kernel.
+// n*C/8 elements of each token's n*C row.
+//
+// Ring stage (one 64-channel block cb of the tile), per pair of streams
+// (2p, 2p+1):  [ phiT rows of stream 2p | of stream 2p+1 ]  (2R rows)
+//              [ X rows of stream 2p (Mt) | of stream 2p+1 (Mt) | unused ]  (128 rows)
+// every row 128 bytes with the 128-byte swizzle.  One MMA per 16-wide K step
+// and pair, D[128 x (2R+128)] += A * B^T with A = the pair's 128 X rows and
+// B = the whole pair region, yields both products the coefficients need:
+// columns [0, 2R) are the projections through phi (a row of stream 2p lands
+// in columns [0, R), of stream 2p+1 in [R, 2R)), and column 2R+m is the dot
+// product of X rows m and m, i.e. row m's sum of squares (Eq.15).  The pairs
+// accumulate into the same columns, so after the tile TMEM row m < Mt holds
+// the sums over streams 0, 2 of token m and row Mt+m those over streams 1, 3.
+// phiT is streamed with X (it stays in L2), which leaves room for 4 stages.
+// An odd n reads a zero-filled last stream (out of the tensor maps' range).
 //
 // Warp roles (16 warps):
-//   0      TMA producer: X[tile, stream i, 64-channel block] boxes (Mt rows x
-//          128 B, 128-byte swizzle, L2 evict-last) through a 14-stage ring;
-//          it runs at most LAG tiles ahead of the x_in warps, which keeps the
-//          x_in re-read inside L2.
-//   1      MMA issuer: D[128 x NB] += X_chunk[128 x 64] * phiT_chunk[NB x 64]^T
-//          and S[128 x 64] += X_chunk * X_chunk[0..63]^T, whose diagonal is
-//          each row's sum of squares (Eq.15) (tcgen05.mma kind::f16, fp32
-//          accumulators in TMEM, double-buffered across tiles; rows >= Mt are
-//          never read).  The MMA commit is the only consumer of a ring stage.
-//   4-5    epilogue: each tile row's partial (logits, sum of squares) from TMEM
-//          is pushed with st.async into the shared memory of the CTA that owns
-//          the token (8 tokens per CTA); the owner reduces the 8 partial rows,
-//          computes the coefficients (Eq.16-19, Sinkhorn in registers) and
-//          pushes H_pre to every CTA of the cluster.  The pushes
-//          complete transactions on the receivers' mbarriers, so no fence or
-//          remote arrive sits on this path.
-//   2-3, 6-15  x_in = H_pre X for this CTA's channels, re-reading the tile's
+//   0      TMA producer: per stage and pair, a {64, R, 2} box of phiT and a
+//          {64, Mt, 2} box of X (L2 evict-last); it runs at most LAG tiles
+//          ahead of the x_in warps, which keeps the x_in re-read in L2.
+//   1      MMA issuer (tcgen05.mma kind::f16, fp32 accumulators in TMEM,
+//          double-buffered across tiles).  The MMA commit is the only
+//          consumer of a ring stage.
+//   4-7    epilogue, one TMEM lane quarter each: every TMEM row (a token's
+//          half: its projections and sum of squares) is pushed with st.async
+//          into the shared memory of the CTA that owns the token (8 tokens per
+//          CTA); warps 4-5 of the owner reduce the 2 x 8 partial rows, compute
+//          the coefficients (Eq.16-19, Sinkhorn in registers) and push H_pre
+//          to every CTA of the cluster.  The pushes complete transactions on
+//          the receivers' mbarriers, so no fence or remote arrive sits on this
+//          path.
+//   2-3, 8-15  x_in = H_pre X for this CTA's channels, re-reading the tile's
 //          X slice from L2 (evict-first on this last read).
 // The roles meet only through mbarriers and one progress counter, so the TMA
 // ring keeps streaming while a tile's coefficients and x_in are produced.
 //
 // HBM: X is read once; x_in and the coefficients are written once; phi is
-// read once per CTA.  Every wait is bounded (g_wait_limit); on expiry the
-// kernel records the timeout in the device error word, drains its own copies
-// and MMAs in flight, frees TMEM and returns.
+// read from HBM about once (its re-reads hit L2).  Every wait is bounded
+// (g_wait_limit); on expiry the kernel records the timeout in the device
+// error word, drains its own copies and MMAs in flight, frees TMEM and returns.
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
@@ -43,54 +54,85 @@ namespace pretc {
 using namespace sm100;
 
 constexpr int CL = 8;            // CTAs per cluster (channel split)
-constexpr int MROWS = 128;       // MMA M (TMEM lanes); a tile uses the first Mt <= MT_CAP rows
+constexpr int MROWS = 128;       // MMA M (TMEM lanes): two streams of up to MT_CAP tokens
 constexpr int MT_CAP = 64;       // token rows per tile: bounds the L2 footprint of the x_in re-read
-constexpr int KC = 64;           // K elements per chunk (one 128-byte row)
-constexpr int STAGE_BYTES = MT_CAP * 128;
-constexpr int STAGES = 14;
+constexpr int KC = 64;           // channels per block (one 128-byte row)
+constexpr int MAX_STAGES = 6;
+constexpr int SMEM_LIMIT = 227 * 1024;
 constexpr int NTHREADS = 512;
-constexpr int EPI_WARP0 = 4, EPI_WARPS = 2, EPI_THREADS = 64;   // TMEM lane quarters 0 and 1
-constexpr int XIN_WARPS = 12, XIN_THREADS = 384;                 // warps 2-3 and 6-15
+constexpr int EPI_WARP0 = 4, EPI_WARPS = 4;                       // TMEM lane quarters 0-3
+constexpr int XIN_WARPS = 10, XIN_THREADS = XIN_WARPS * 32;       // warps 2-3 and 8-15
 constexpr int TOK_PER_CTA = MT_CAP / CL;  // tokens whose coefficients a CTA computes
 constexpr int XIN_UNROLL = 4;             // x_in vectors in flight per thread
-constexpr int LAG = 2;                    // tiles the TMA stream may run ahead of x_in
-static_assert(TOK_PER_CTA * 8 <= EPI_THREADS, "one 8-lane group per coefficient token");
+#ifndef MHC_PRE_LAG
+#define MHC_PRE_LAG 2
+#endif
+constexpr int LAG = MHC_PRE_LAG;          // tiles the TMA stream may run ahead of x_in
+constexpr int ACC_COLS = 256;             // TMEM columns per accumulator buffer
+constexpr int TMEM_COLS = 512;
+static_assert(TOK_PER_CTA * 8 == 64, "warps 4-5: one 8-lane group per coefficient token");
 
 template <int N> struct Cfg {
     static constexpr int P = N * N + 2 * N;
-    static constexpr int R = (P + 7) / 8 * 8;      // phiT rows stored per chunk
-    static constexpr int NB = (P + 15) / 16 * 16;  // MMA N
-    static constexpr int PS = P + 1;               // partial row: P logits + sum of squares
-    static constexpr int PSP = (PS + 3) / 4 * 4;   // ... padded to 16-byte multiples
-    static constexpr int SQ_COL = 2 * NB;           // X X^T accumulators (2 x MT_CAP columns) after the logits
-    static constexpr int TMEM_COLS = 256;
+    static constexpr int R = (P + 7) / 8 * 8;       // phiT rows per stream in a stage
+    static constexpr int NP = (N + 1) / 2;          // stream pairs
+    static constexpr int MMA_N = 2 * R + MROWS;     // B rows: the pair's phiT rows, then its X rows
+    static constexpr int PAIR_BYTES = MMA_N * 128;
+    static constexpr int STAGE_BYTES = NP * PAIR_BYTES;
+    static constexpr int PS = P + 1;                // partial row: P projections + sum of squares
+    static constexpr int PSP = (PS + 3) / 4 * 4;    // ... padded to 16-byte multiples
+    static_assert(MMA_N % 16 == 0 && MMA_N <= ACC_COLS, "MMA N for M = 128");
 };
 
-enum Bar { B_FULL = 0, B_EMPTY = B_FULL + STAGES, B_TFULL = B_EMPTY + STAGES, B_TEMPTY = B_TFULL + 2,
-           B_PART = B_TEMPTY + 2, B_HPRE, B_XIN = B_HPRE + 2, B_PHI, B_DRAIN, B_COUNT };
+enum Bar { B_FULL = 0, B_EMPTY = B_FULL + MAX_STAGES, B_TFULL = B_EMPTY + MAX_STAGES, B_TEMPTY = B_TFULL + 2,
+           B_PART = B_TEMPTY + 2, B_HPRE, B_XIN = B_HPRE + 2, B_DRAIN, B_COUNT };
 
 struct Layout {
-    uint32_t phi, ring, part, hpre, bias, bars, slot, total;
+    uint32_t ring, part, hpre, bias, bars, slot, total;
+    int stages;
 };
 
+// Bytes after the ring: partial rows [CL][2 halves][TOK_PER_CTA][PSP], H_pre
+// [2][MT_CAP][N], b, barriers.
 template <int N>
-__host__ __device__ inline Layout layout_for(int NQ) {
+__host__ __device__ constexpr uint32_t layout_fixed_bytes() {
+    using G = Cfg<N>;
+    return CL * 2 * TOK_PER_CTA * G::PSP * 4 + 2 * MT_CAP * N * 4 + G::P * 4 + 16 + B_COUNT * 8 + 16;
+}
+
+// Shared memory plan: the ring takes as many stages (up to MAX_STAGES) as the
+// rest of the 227 KB leaves room for.
+template <int N>
+__host__ __device__ inline Layout layout_for() {
     using G = Cfg<N>;
     Layout L;
-    L.phi = 0;
-    L.ring = uint32_t(NQ) * G::R * 128;                      // multiple of 1024
-    L.part = L.ring + STAGES * STAGE_BYTES;
-    L.hpre = L.part + CL * TOK_PER_CTA * G::PSP * 4;       // after [source CTA][token][PSP]
+    L.ring = 0;
+    {
+        const int64_t room = int64_t(SMEM_LIMIT) - 1024 - layout_fixed_bytes<N>();
+        const int64_t fit = room > 0 ? room / G::STAGE_BYTES : 0;
+        L.stages = int(fit < MAX_STAGES ? fit : MAX_STAGES);
+    }
+    L.part = L.ring + uint32_t(L.stages) * G::STAGE_BYTES;
+    L.hpre = L.part + CL * 2 * TOK_PER_CTA * G::PSP * 4;
     L.bias = L.hpre + 2 * MT_CAP * N * 4;
     L.bars = (L.bias + G::P * 4 + 15) / 16 * 16;
     L.slot = L.bars + B_COUNT * 8;
     L.total = L.slot + 16;
-    // The MMA reads 128 rows from a stage's base: the last stage's rows past
-    // MT_CAP must still be inside this CTA's shared memory (their products land
-    // in accumulator rows that are never read).
-    const uint32_t mma_end = L.part + (MROWS - MT_CAP) * 128;
-    if (L.total < mma_end) L.total = mma_end;
     return L;
+}
+
+// TMEM row r of a tile -> (half h, token) for rows r < 2 Mt; the unused rows
+// r >= 2 Mt map one-to-one onto the slots of tokens Mt..MT_CAP-1, so that every
+// owner receives the same number of bytes for every tile.
+__device__ __forceinline__ void row_slot(int r, int Mt, int& h, int& tok) {
+    if (r < 2 * Mt) {
+        h = r >= Mt ? 1 : 0;
+        tok = r - h * Mt;
+    } else {
+        const int k = r - 2 * Mt, spare = MT_CAP - Mt;     // spare >= 1 here
+        h = k / spare;
+        tok = Mt + k % spare;
+    }
 }
 
 template <int N>
@@ -103,18 +145,18 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
               float* __restrict__ r_out)
 {
     using G = Cfg<N>;
-    constexpr int P = G::P, R = G::R, NB = G::NB, PS = G::PS, PSP = G::PSP;
+    constexpr int P = G::P, R = G::R, NP = G::NP, PS = G::PS, PSP = G::PSP;
+    constexpr int STAGE_BYTES = G::STAGE_BYTES, PAIR_BYTES = G::PAIR_BYTES;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte-swizzle atoms
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int Cs = C / CL;
-    const int CB = Cs / KC;            // channel blocks per stream
-    const int NQ = N * CB;             // K chunks of this CTA per tile
-    const Layout L = layout_for<N>(NQ);
-    uint8_t* sphi = smem + L.phi;
+    const int CB = Cs / KC;            // channel blocks = ring stages per tile
+    const Layout L = layout_for<N>();
+    const int STAGES = L.stages;
     uint8_t* sring = smem + L.ring;
-    float* rpart = reinterpret_cast<float*>(smem + L.part);   // [CL][TOK_PER_CTA][PSP], pushed by the cluster
+    float* rpart = reinterpret_cast<float*>(smem + L.part);   // [CL][2][TOK_PER_CTA][PSP], pushed by the cluster
     float* shpre = reinterpret_cast<float*>(smem + L.hpre);   // [2][MT_CAP][N]
     float* sb = reinterpret_cast<float*>(smem + L.bias);      // b, kept on chip for the coefficients
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
@@ -122,10 +164,9 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     uint64_t* empty = bars + B_EMPTY;
     uint64_t* tfull = bars + B_TFULL;
     uint64_t* tempty = bars + B_TEMPTY;
-    uint64_t* part_full = bars + B_PART;     // this CTA's tokens: all CL partial rows landed
+    uint64_t* part_full = bars + B_PART;     // this CTA's tokens: all partial rows landed
     uint64_t* hpre_full = bars + B_HPRE;     // [2] H_pre of every tile row landed (per tile parity)
     uint64_t* xin_prog = bars + B_XIN;
-    uint64_t* phi_full = bars + B_PHI;
     uint64_t* drain = bars + B_DRAIN;
     uint32_t* slot = reinterpret_cast<uint32_t*>(smem + L.slot);
     __shared__ int s_abort;
@@ -154,11 +195,10 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         mbar_init(&hpre_full[0], 1);
         mbar_init(&hpre_full[1], 1);
         mbar_init(xin_prog, XIN_WARPS);
-        mbar_init(phi_full, 1);
         mbar_init(drain, 1);
         fence_mbar_init();
     }
-    if (warp == 1) tmem_alloc(slot, G::TMEM_COLS);
+    if (warp == 1) tmem_alloc(slot, TMEM_COLS);
     for (int p = threadIdx.x; p < P; p += NTHREADS) sb[p] = b[p];
     __syncthreads();
     tc_fence_after();
@@ -166,11 +206,6 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     if (threadIdx.x == 0) {
         tma_prefetch(&tmX);
         tma_prefetch(&tmPhi);
-        // Resident phiT: chunk q = (stream i, channel block cb) holds rows p < R of
-        // phiT[p][i*C + c0 + cb*64 + 0..63] (rows >= P are zero-filled by the TMA).
-        mbar_arrive_expect_tx(phi_full, uint32_t(NQ) * R * 128);
-        for (int q = 0; q < NQ; ++q)
-            tma_load_2d(sphi + size_t(q) * R * 128, &tmPhi, phi_full, (q / CB) * C + c0 + (q % CB) * KC, 0);
     }
     cluster_sync();   // every CTA's barriers are initialised before any remote arrive
 
@@ -178,9 +213,10 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             const uint64_t keep = policy_evict_last();
+            const uint32_t stage_tx = uint32_t(NP) * uint32_t(2 * R + 2 * Mt) * 128;
             int s = 0;
             uint32_t ph = 0;
-            int inflight_s[STAGES], inflight_ph[STAGES], n_issued = 0;
+            int inflight_s[MAX_STAGES], inflight_ph[MAX_STAGES], n_issued = 0;
             bool ok = true;
             int it = 0;
             for (int tile = cluster_id; tile < num_tiles && ok; tile += nclusters, ++it) {
@@ -195,50 +231,60 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     }
                     if (k >= g_wait_limit) { atomicOr(&g_device_error, 1u); ok = false; break; }
                 }
-                for (int q = 0; q < NQ; ++q) {
+                for (int cb = 0; cb < CB; ++cb) {
                     if (!mbar_wait(&empty[s], ph ^ 1) || *(volatile int*)&s_abort) { ok = false; break; }
-                    mbar_arrive_expect_tx(&full[s], uint32_t(Mt) * 128);
-                    tma_load_3d_hint(sring + s * STAGE_BYTES, &tmX, &full[s], c0 + (q % CB) * KC, q / CB, t0, keep);
-                    inflight_s[n_issued % STAGES] = s;
-                    inflight_ph[n_issued % STAGES] = int(ph);
+                    mbar_arrive_expect_tx(&full[s], stage_tx);
+                    const int cc = c0 + cb * KC;
+#pragma unroll
+                    for (int p = 0; p < NP; ++p) {
+                        uint8_t* pb = sring + s * STAGE_BYTES + p * PAIR_BYTES;
+                        // phiT {64 channels, R rows, streams 2p..2p+1} of the {C, P, n} view
+                        tma_load_3d_hint(pb, &tmPhi, &full[s], cc, 0, 2 * p, keep);
+                        // X {64 channels, Mt tokens, streams 2p..2p+1} of the {C, T, n} view
+                        tma_load_3d_hint(pb + 2 * R * 128, &tmX, &full[s], cc, t0, 2 * p, keep);
+                    }
+                    inflight_s[n_issued % MAX_STAGES] = s;
+                    inflight_ph[n_issued % MAX_STAGES] = int(ph);
                     ++n_issued;
                     if (++s == STAGES) { s = 0; ph ^= 1; }
                 }
             }
             if (!ok) {
                 s_abort = 1;
-                // drain this CTA's copies still in flight before the block can exit
+                // drain this CTA's copies still in flight (the ring slots of the
+                // last min(n_issued, STAGES) stages) before the block can exit
                 const int pending = n_issued < STAGES ? n_issued : STAGES;
-                for (int j = 0; j < pending; ++j)
-                    mbar_wait(&full[inflight_s[j]], uint32_t(inflight_ph[j]), 1ll << 22);
+                for (int j = 0; j < pending; ++j) {
+                    const int k = (n_issued - 1 - j) % MAX_STAGES;
+                    mbar_wait(&full[inflight_s[k]], uint32_t(inflight_ph[k]), 1ll << 22);
+                }
             }
         }
-        if (lane == 1) mbar_wait(phi_full, 0, 1ll << 24);     // phiT copy settles before any exit
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(MROWS, NB);
-            constexpr uint32_t idesc_sq = idesc_bf16_f32(MROWS, MT_CAP);   // X X^T, tile rows only
-            const uint32_t ring_a = smem_u32(sring), phi_a = smem_u32(sphi);
+            constexpr uint32_t idesc = idesc_bf16_f32(MROWS, G::MMA_N);
+            const uint32_t ring_a = smem_u32(sring);
             int s = 0, it = 0;
             uint32_t ph = 0;
-            bool ok = mbar_wait(phi_full, 0);
+            bool ok = true;
             for (int tile = cluster_id; tile < num_tiles && ok; tile += nclusters, ++it) {
                 const int acc = it & 1;
                 if (!mbar_wait(&tempty[acc], (uint32_t((it >> 1) & 1)) ^ 1)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d = tmem_base + uint32_t(acc * NB);
-                const uint32_t dsq = tmem_base + uint32_t(G::SQ_COL + acc * MT_CAP);
-                for (int q = 0; q < NQ; ++q) {
+                const uint32_t d = tmem_base + uint32_t(acc * ACC_COLS);
+                for (int cb = 0; cb < CB; ++cb) {
                     if (!mbar_wait(&full[s], ph) || *(volatile int*)&s_abort) { ok = false; break; }
                     tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < KC / 16; ++kk) {
-                        const uint64_t ad = sdesc_k_sw128(ring_a + s * STAGE_BYTES + kk * 32);
-                        const uint64_t bd = sdesc_k_sw128(phi_a + q * R * 128 + kk * 32);
-                        mma_bf16(d, ad, bd, idesc, (q | kk) != 0);
-                        // Eq.(15): the sums of squares are the diagonal of X X^T (B = the same rows)
-                        mma_bf16(dsq, ad, ad, idesc_sq, (q | kk) != 0);
+                    for (int p = 0; p < NP; ++p) {
+#pragma unroll
+                        for (int kk = 0; kk < KC / 16; ++kk) {
+                            const uint32_t pb = ring_a + s * STAGE_BYTES + p * PAIR_BYTES + kk * 32;
+                            const uint64_t ad = sdesc_k_sw128(pb + 2 * R * 128);   // the pair's X rows
+                            const uint64_t bd = sdesc_k_sw128(pb);                 // phiT rows, then X rows
+                            mma_bf16(d, ad, bd, idesc, (cb | p | kk) != 0);
+                        }
                     }
                     mma_commit(&empty[s]);
                     if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -252,17 +298,20 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             }
         }
 
-    } else if (warp == EPI_WARP0 || warp == EPI_WARP0 + 1) {
+    } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + EPI_WARPS) {
         // ------------------------------------------------------------ epilogue
-        const int et = threadIdx.x - EPI_WARP0 * 32;    // 0..63
-        const int qd = warp & 3;                        // TMEM lane quarter of this warp (0, 1)
-        const int m = qd * 32 + lane;                   // token row within the tile
+        const int et = threadIdx.x - EPI_WARP0 * 32;    // 0..127
+        const int qd = warp & 3;                        // TMEM lane quarter of this warp
+        const int r = qd * 32 + lane;                   // TMEM row (lane)
         const float inv_K = 1.0f / float(N * C);
-        constexpr uint32_t PART_BYTES = CL * TOK_PER_CTA * PSP * 4;
+        constexpr uint32_t PART_BYTES = CL * 2 * TOK_PER_CTA * PSP * 4;
         constexpr uint32_t HPRE_BYTES = MT_CAP * N * 4;
-        // the partial row of tile row m goes to its owner CTA m / TOK_PER_CTA, slot (rank, m % TOK_PER_CTA)
-        const uint32_t owner = uint32_t(m / TOK_PER_CTA);
-        const uint32_t push_dst = mapa(smem_u32(rpart + (int(rank) * TOK_PER_CTA + m % TOK_PER_CTA) * PSP), owner);
+        int h, tok;
+        row_slot(r, Mt, h, tok);
+        // the partial row goes to the token's owner CTA, slot (rank, half, token % TOK_PER_CTA)
+        const uint32_t owner = uint32_t(tok / TOK_PER_CTA);
+        const uint32_t push_dst =
+            mapa(smem_u32(rpart + ((int(rank) * 2 + h) * TOK_PER_CTA + tok % TOK_PER_CTA) * PSP), owner);
         const uint32_t push_bar = mapa(smem_u32(part_full), owner);
         int it = 0;
         for (int tile = cluster_id; tile < num_tiles; tile += nclusters, ++it) {
@@ -276,28 +325,24 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             }
             if (!mbar_wait(&tfull[acc], par)) { s_abort = 1; break; }
             tc_fence_after();
-            float d[NB];
-            const uint32_t taddr = tmem_base + (uint32_t(qd * 32) << 16) + uint32_t(acc * NB);
+            float d[2 * R];
+            const uint32_t taddr = tmem_base + (uint32_t(qd * 32) << 16) + uint32_t(acc * ACC_COLS);
 #pragma unroll
-            for (int c = 0; c < NB; c += 16) {
+            for (int c = 0; c < 2 * R; c += 16) {
                 float tmp[16];
                 tmem_ld16(taddr + c, tmp);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) d[c + j] = tmp[j];
+                for (int j = 0; j < 16; ++j) if (c + j < 2 * R) d[c + j] = tmp[j];
             }
             float ss = 0.0f;
-            {
-                const uint32_t qaddr = tmem_base + (uint32_t(qd * 32) << 16) +
-                                       uint32_t(G::SQ_COL + acc * MT_CAP + qd * 32);
 #pragma unroll
-                for (int c = 0; c < 32; c += 16) {
-                    float tmp[16];
-                    tmem_ld16(qaddr + c, tmp);
-                    tmem_wait_ld();
+            for (int c = 0; c < 32; c += 16) {          // column 2R + r: X row r . X row r
+                float tmp[16];
+                tmem_ld16(taddr + 2 * R + qd * 32 + c, tmp);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) if (c + j == lane) ss = tmp[j];   // diagonal (m, m)
-                }
+                for (int j = 0; j < 16; ++j) if (c + j == lane) ss = tmp[j];
             }
             tc_fence_before();
             __syncwarp();
@@ -306,30 +351,32 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             // H_pre of tile it lands in buffer it&1, last read by the x_in warps for
             // tile it-2: they must have moved on (they arrive after their tile it-1 wait)
             if (it >= 1 && !mbar_wait(xin_prog, uint32_t((it - 1) & 1))) { s_abort = 1; break; }
-            // push (partial logits, sum of squares) of row m to its owner
+            // push (partial projections, sum of squares) of this row's half to its owner
 #pragma unroll
             for (int p = 0; p < PSP; p += 4) {
-                float4 w4;
-                w4.x = p + 0 < P ? d[p + 0] : (p + 0 == P ? ss : 0.0f);
-                w4.y = p + 1 < P ? d[p + 1] : (p + 1 == P ? ss : 0.0f);
-                w4.z = p + 2 < P ? d[p + 2] : (p + 2 == P ? ss : 0.0f);
-                w4.w = p + 3 < P ? d[p + 3] : (p + 3 == P ? ss : 0.0f);
-                st_async_f32x4(push_dst + p * 4, w4, push_bar);
+                float w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int q = p + e;
+                    w[e] = q < P ? (h ? d[R + q] : d[q]) : (q == P ? ss : 0.0f);   // q < P <= R
+                }
+                st_async_f32x4(push_dst + p * 4, make_float4(w[0], w[1], w[2], w[3]), push_bar);
             }
-            if (!mbar_wait(part_full, uint32_t(it & 1))) { s_abort = 1; break; }
-
-            // Coefficients of this CTA's TOK_PER_CTA tokens: a group of 8 lanes per
-            // token; lane g takes the partial row from CTA g, the group reduces, then
-            // lane g < N carries row g of H_res through a row-parallel Sinkhorn.
-            {
+            if (et < 64) {
+                if (!mbar_wait(part_full, uint32_t(it & 1))) { s_abort = 1; break; }
+                // Coefficients of this CTA's TOK_PER_CTA tokens: a group of 8 lanes per
+                // token; lane g adds the two half rows from CTA g, the group reduces,
+                // then lane g < N carries row g of H_res through the Sinkhorn.
                 const int jj = et >> 3, g = et & 7;
                 const int j = int(rank) * TOK_PER_CTA + jj;     // row within the tile
-                const float* src = rpart + (g * TOK_PER_CTA + jj) * PSP;
+                const float* src0 = rpart + ((g * 2 + 0) * TOK_PER_CTA + jj) * PSP;
+                const float* src1 = rpart + ((g * 2 + 1) * TOK_PER_CTA + jj) * PSP;
                 float v[PSP];
 #pragma unroll
                 for (int p = 0; p < PSP; p += 4) {
-                    const float4 f4 = *reinterpret_cast<const float4*>(src + p);
-                    v[p] = f4.x; v[p + 1] = f4.y; v[p + 2] = f4.z; v[p + 3] = f4.w;
+                    const float4 f0 = *reinterpret_cast<const float4*>(src0 + p);
+                    const float4 f1 = *reinterpret_cast<const float4*>(src1 + p);
+                    v[p] = f0.x + f1.x; v[p + 1] = f0.y + f1.y; v[p + 2] = f0.z + f1.z; v[p + 3] = f0.w + f1.w;
                 }
 #pragma unroll
                 for (int p = 0; p < PS; ++p) {
@@ -337,8 +384,8 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     v[p] += __shfl_xor_sync(0xffffffffu, v[p], 2);
                     v[p] += __shfl_xor_sync(0xffffffffu, v[p], 4);
                 }
-                const float r = sqrtf(v[P] * inv_K + eps);                     // Eq.(15)
-                const float inv_r = 1.0f / r;
+                const float rr_ = sqrtf(v[P] * inv_K + eps);                   // Eq.(15)
+                const float inv_r = 1.0f / rr_;
                 // every lane of the group carries the whole n x n Sinkhorn (no shuffles in
                 // the iterations); lane g < N then keeps stream g's gates and H_res row g
                 float mres[N][N];
@@ -364,7 +411,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     // every CTA needs H_pre of every tile row for its x_in channels
                     const uint32_t hoff = smem_u32(shpre + (acc * MT_CAP + j) * N + g);
                     const uint32_t hbar = smem_u32(&hpre_full[acc]);
-                    for (uint32_t rr = 0; rr < CL; ++rr) st_async_f32(mapa(hoff, rr), hp, mapa(hbar, rr));
+                    for (uint32_t cr = 0; cr < CL; ++cr) st_async_f32(mapa(hoff, cr), hp, mapa(hbar, cr));
                     const int64_t t = t0 + j;
                     if (j < Mt && t < T) {
                         if (Hpost) Hpost[t * N + g] = 2.0f * sigmoidf_(zpost);     // Eq.(18)
@@ -379,7 +426,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
 #pragma unroll
                     for (int p = 0; p < P; ++p)
                         if ((p & 7) == g) u_out[(t0 + j) * P + p] = v[p] * inv_r;
-                    if (g == 0) r_out[t0 + j] = r;
+                    if (g == 0) r_out[t0 + j] = rr_;
                 }
             }
             // every owner has read its partial rows of this tile once this CTA holds the
@@ -388,7 +435,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         }
     } else {
         // ------------------------------------------------------------ x_in
-        const int xt = (warp < EPI_WARP0 ? warp - 2 : warp - 4) * 32 + lane;   // 0..XIN_THREADS-1
+        const int xt = (warp < EPI_WARP0 ? warp - 2 : warp - (EPI_WARP0 + EPI_WARPS - 2)) * 32 + lane;
         const uint64_t drop = policy_evict_first();
         const int VPT = Cs / 8;                          // 16-byte vectors per token
         int it = 0;
@@ -402,16 +449,16 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             const int items = x_in ? rows * VPT : 0;
             for (int w0 = xt; w0 < items; w0 += XIN_UNROLL * XIN_THREADS) {
                 uint4 raw[XIN_UNROLL][N];
-                int tok[XIN_UNROLL], cc[XIN_UNROLL];
+                int tk[XIN_UNROLL], cc[XIN_UNROLL];
 #pragma unroll
                 for (int u = 0; u < XIN_UNROLL; ++u) {
                     const int w = w0 + u * XIN_THREADS;
                     const int wc = w < items ? w : items - 1;   // clamp; the store is skipped
-                    tok[u] = wc / VPT;
-                    cc[u] = c0 + (wc - tok[u] * VPT) * 8;
+                    tk[u] = wc / VPT;
+                    cc[u] = c0 + (wc - tk[u] * VPT) * 8;
 #pragma unroll
                     for (int i = 0; i < N; ++i)
-                        raw[u][i] = ldg16_raw_hint(X + ((t0 + tok[u]) * N + i) * C + cc[u], drop);
+                        raw[u][i] = ldg16_raw_hint(X + ((t0 + tk[u]) * N + i) * C + cc[u], drop);
                 }
 #pragma unroll
                 for (int u = 0; u < XIN_UNROLL; ++u) {
@@ -421,15 +468,15 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     for (int e = 0; e < 8; ++e) o[e] = 0.0f;
 #pragma unroll
                     for (int i = 0; i < N; ++i) {
-                        const float h = hb[tok[u] * N + i];
+                        const float hh = hb[tk[u] * N + i];
                         const uint32_t w4[4] = {raw[u][i].x, raw[u][i].y, raw[u][i].z, raw[u][i].w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            o[2 * e] = fmaf(h, bf16_lo(w4[e]), o[2 * e]);
-                            o[2 * e + 1] = fmaf(h, bf16_hi(w4[e]), o[2 * e + 1]);
+                            o[2 * e] = fmaf(hh, bf16_lo(w4[e]), o[2 * e]);
+                            o[2 * e + 1] = fmaf(hh, bf16_hi(w4[e]), o[2 * e + 1]);
                         }
                     }
-                    store16<false>(x_in + (t0 + tok[u]) * C + cc[u], o);
+                    store16<false>(x_in + (t0 + tk[u]) * C + cc[u], o);
                 }
             }
             __syncwarp();
@@ -440,7 +487,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, G::TMEM_COLS);
+        tmem_dealloc(tmem_base, TMEM_COLS);
     }
     cluster_sync();   // no CTA leaves while a peer may still touch its shared memory
 }
@@ -466,17 +513,20 @@ static EncodeTiledFn encode_fn()
 }
 
 template <int N>
-static int smem_bytes(int C) { return int(layout_for<N>(N * (C / CL) / KC).total) + 1024; }
+static int smem_bytes() { return int(layout_for<N>().total) + 1024; }
 
 template <int N>
-static bool fits(int C) { return C % (CL * KC) == 0 && smem_bytes<N>(C) <= 227 * 1024; }
+static bool fits(int C)
+{
+    return C % (CL * KC) == 0 && layout_for<N>().stages >= 2 && smem_bytes<N>() <= SMEM_LIMIT;
+}
 
 template <int N>
 static mhc_status launch_n(const PreArgs& a, cudaStream_t s)
 {
     static int configured_smem = 0;
     static int max_clusters = 0;
-    const int smem = smem_bytes<N>(a.C);
+    const int smem = smem_bytes<N>();
     auto kern = pre_tc_kernel<N>;
     if (smem > configured_smem) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -499,11 +549,19 @@ static mhc_status launch_n(const PreArgs& a, cudaStream_t s)
                                                              "mhc_pre (tc): cluster occupancy");
         max_clusters = nc;
     }
-    // Token tiles of Mt <= 128 rows, sized so that every cluster gets the same number.
-    const int64_t rounds = (a.T + int64_t(max_clusters) * MT_CAP - 1) / (int64_t(max_clusters) * MT_CAP);
-    const int64_t per_round = (a.T + rounds - 1) / rounds;                     // tokens per round
-    int Mt = int((per_round + max_clusters - 1) / max_clusters);
-    if (Mt > MT_CAP) Mt = MT_CAP;
+    // Token tiles of Mt rows, Mt a multiple of 8 (each stream's rows in a stage
+    // then start on a 1024-byte swizzle atom) and at most MT_CAP.  A tile costs
+    // its Mt tokens plus a fixed overhead worth about TILE_COST tokens (the MMAs
+    // always cover 128 rows; the coefficient exchange; a shorter TMA box); take
+    // the Mt that minimises the busiest cluster's cost (ties: the larger Mt).
+    constexpr int TILE_COST = 32;
+    int Mt = MT_CAP;
+    int64_t best = -1;
+    for (int m = MT_CAP; m >= 8; m -= 8) {
+        const int64_t tiles = (a.T + m - 1) / m;
+        const int64_t cost = (tiles + max_clusters - 1) / max_clusters * (m + TILE_COST);
+        if (best < 0 || cost < best) { best = cost; Mt = m; }
+    }
     const int64_t tiles64 = (a.T + Mt - 1) / Mt;
     const int nclusters = int(tiles64 < max_clusters ? tiles64 : max_clusters);
 
@@ -515,9 +573,11 @@ static mhc_status launch_n(const PreArgs& a, cudaStream_t s)
     using G = Cfg<N>;
     CUtensorMap mapX, mapPhi;
     {
-        const cuuint64_t dims[3] = {cuuint64_t(a.C), cuuint64_t(a.n), cuuint64_t(a.T)};
-        const cuuint64_t strides[2] = {cuuint64_t(a.C) * 2, cuuint64_t(a.n) * a.C * 2};
-        const cuuint32_t box[3] = {KC, 1, cuuint32_t(Mt)};
+        // X [T][n][C] viewed as {C, T, n}: a box {64, Mt, 2} lands stream-major
+        // (the Mt rows of stream 2p, then those of stream 2p+1)
+        const cuuint64_t dims[3] = {cuuint64_t(a.C), cuuint64_t(a.T), cuuint64_t(a.n)};
+        const cuuint64_t strides[2] = {cuuint64_t(a.n) * a.C * 2, cuuint64_t(a.C) * 2};
+        const cuuint32_t box[3] = {KC, cuuint32_t(Mt), 2};
         const cuuint32_t estr[3] = {1, 1, 1};
         CUresult r = enc(&mapX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.X), dims, strides,
                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -528,12 +588,13 @@ static mhc_status launch_n(const PreArgs& a, cudaStream_t s)
         }
     }
     {
-        const cuuint64_t K = cuuint64_t(a.n) * a.C;
-        const cuuint64_t dims[2] = {K, cuuint64_t(G::P)};
-        const cuuint64_t strides[1] = {K * 2};
-        const cuuint32_t box[2] = {KC, cuuint32_t(G::R)};
-        const cuuint32_t estr[2] = {1, 1};
-        CUresult r = enc(&mapPhi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.phi), dims, strides,
+        // phiT [P][n*C] viewed as {C, P, n}: a box {64, R, 2} holds the R rows
+        // (rows >= P zero-filled) of streams 2p and 2p+1 for one channel block
+        const cuuint64_t dims[3] = {cuuint64_t(a.C), cuuint64_t(G::P), cuuint64_t(a.n)};
+        const cuuint64_t strides[2] = {cuuint64_t(a.n) * a.C * 2, cuuint64_t(a.C) * 2};
+        const cuuint32_t box[3] = {KC, cuuint32_t(G::R), 2};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        CUresult r = enc(&mapPhi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.phi), dims, strides,
                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) {
