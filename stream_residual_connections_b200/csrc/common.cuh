@@ -68,14 +68,23 @@ __device__ __forceinline__ float to_f32(bf16_t v) { return __uint_as_float(uint3
 
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + expf(-z)); }
 
+// Approximate reciprocal: the PTX rcp.approx.ftz.f32 instruction (at most 1 ulp
+// from 1/x for normal x, per the PTX ISA).  Operands here are sums of positive
+// values of order one, far from the subnormal range that ftz flushes.
+__device__ __forceinline__ float fast_rcp(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 // Sinkhorn-Knopp on an N x N logit matrix held in registers ([mHC] Eq.(8)-(9)):
 // M = exp(L); `iters` times normalise every column, then every row.  Each
 // column is shifted by its maximum before exp when iters >= 1; the first
 // column normalisation cancels any per-column factor, so the result is the
-// same and exp cannot overflow.  The normalisers use the fast reciprocal
-// (__fdividef, within 2 ulp): a correctly rounded reciprocal is a long
-// dependent sequence on this GPU (measured ~4x slower for 20 iterations), and
-// the coefficients are only required to 1e-5.
+// same and exp cannot overflow.  The iterations form one dependent chain, so
+// the normalisers use the approximate reciprocal: a correctly rounded one is
+// a long sequence on this GPU (20 iterations measured ~4x slower), and the
+// coefficients are only required to 1e-5.
 template <int N>
 __device__ __forceinline__ void sinkhorn_regs(float (&m)[N][N], int iters) {
 #pragma unroll
@@ -93,7 +102,7 @@ __device__ __forceinline__ void sinkhorn_regs(float (&m)[N][N], int iters) {
             float s = 0.0f;
 #pragma unroll
             for (int i = 0; i < N; ++i) s += m[i][j];
-            const float inv = __fdividef(1.0f, s);   // fast reciprocal (<= 2 ulp); see below
+            const float inv = fast_rcp(s);
 #pragma unroll
             for (int i = 0; i < N; ++i) m[i][j] *= inv;
         }
@@ -102,7 +111,7 @@ __device__ __forceinline__ void sinkhorn_regs(float (&m)[N][N], int iters) {
             float s = 0.0f;
 #pragma unroll
             for (int j = 0; j < N; ++j) s += m[i][j];
-            const float inv = __fdividef(1.0f, s);
+            const float inv = fast_rcp(s);
 #pragma unroll
             for (int j = 0; j < N; ++j) m[i][j] *= inv;
         }

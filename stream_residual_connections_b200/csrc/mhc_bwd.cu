@@ -106,7 +106,7 @@ b1_kernel(const TX* __restrict__ X, const TX* __restrict__ F, const TX* __restri
                 float s = 0.0f;
 #pragma unroll
                 for (int i = 0; i < N; ++i) s += m[i][j];
-                const float inv = __fdividef(1.0f, s);
+                const float inv = fast_rcp(s);
 #pragma unroll
                 for (int i = 0; i < N; ++i) m[i][j] *= inv;
             }
@@ -115,7 +115,7 @@ b1_kernel(const TX* __restrict__ X, const TX* __restrict__ F, const TX* __restri
                 float s = 0.0f;
 #pragma unroll
                 for (int j = 0; j < N; ++j) s += m[i][j];
-                const float inv = __fdividef(1.0f, s);
+                const float inv = fast_rcp(s);
 #pragma unroll
                 for (int j = 0; j < N; ++j) m[i][j] *= inv;
             }
@@ -200,7 +200,7 @@ b1_kernel(const TX* __restrict__ X, const TX* __restrict__ F, const TX* __restri
 #pragma unroll
                 for (int i = 0; i < N; ++i) s += Mp[i][j];
                 cs[j] = s;
-                const float inv = __fdividef(1.0f, s);
+                const float inv = fast_rcp(s);
 #pragma unroll
                 for (int i = 0; i < N; ++i) A[i][j] = Mp[i][j] * inv;
             }
@@ -216,7 +216,7 @@ b1_kernel(const TX* __restrict__ X, const TX* __restrict__ F, const TX* __restri
                 float d = 0.0f;
 #pragma unroll
                 for (int j = 0; j < N; ++j) d = fmaf(g[i][j], Mo[i][j], d);
-                const float inv = __fdividef(1.0f, rs[i]);
+                const float inv = fast_rcp(rs[i]);
 #pragma unroll
                 for (int j = 0; j < N; ++j) ga[i][j] = (g[i][j] - d) * inv;
             }
@@ -225,7 +225,7 @@ b1_kernel(const TX* __restrict__ X, const TX* __restrict__ F, const TX* __restri
                 float d = 0.0f;
 #pragma unroll
                 for (int i = 0; i < N; ++i) d = fmaf(ga[i][j], A[i][j], d);
-                const float inv = __fdividef(1.0f, cs[j]);
+                const float inv = fast_rcp(cs[j]);
 #pragma unroll
                 for (int i = 0; i < N; ++i) g[i][j] = (ga[i][j] - d) * inv;
             }

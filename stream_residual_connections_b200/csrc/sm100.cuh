@@ -120,6 +120,16 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) 
     return false;
 }
 
+// Warp-uniform bounded waits: every lane polls and the warp agrees on the
+// outcome, so that a lane whose polls ran out never leaves the others to run a
+// warp-collective instruction (tcgen05.ld, a full-mask shuffle) without it.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+}
+__device__ __forceinline__ bool warp_wait_sleep(uint64_t* bar, uint32_t parity) {
+    return __all_sync(0xffffffffu, mbar_wait_sleep(bar, parity));
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");

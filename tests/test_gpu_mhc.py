@@ -166,10 +166,14 @@ def restore_path():
 
 
 @pytest.mark.parametrize("T,n,C", [(1, 4, 512), (3, 4, 512), (129, 4, 1024), (1000, 2, 512),
-                                   (300, 3, 2048), (257, 4, 4096), (50, 4, 2048), (2500, 4, 1024)])
+                                   (300, 3, 2048), (257, 4, 4096), (50, 4, 2048), (2500, 4, 1024),
+                                   (700, 4, 7168), (333, 3, 7168), (901, 4, 1536), (450, 2, 3072),
+                                   (5000, 4, 4096)])
 def test_tensor_core_path_shapes(T, n, C, restore_path):
-    """TMA + tcgen05 projection (8-CTA clusters): one and several tiles per
-    cluster, ragged last tile, n = 2, 3, 4."""
+    """TMA + tcgen05 projection: one and several tiles per cluster, ragged last
+    tile, n = 2, 3, 4; clusters of 8 CTAs (C = 512, 1536) and of 16 (C a
+    multiple of 1024); phiT resident in the ring (up to 4 channel blocks per
+    CTA) or streamed with X (C = 7168: 7 blocks per CTA)."""
     M.mhc_set_path(M.MHC_PATH_TENSOR)
     inp = synth.mhc_inputs(T, n, C, "bf16", seed=400 + T + n + C)
     _compare(inp, _run(inp))
