@@ -381,6 +381,125 @@ def run_ours(args, world, rank, local):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------- secondary workloads
+def xhc_bytes(T: int, N: int, k: int, m: int, C: int, r: int, kappa_sum: int) -> dict:
+    """Bytes each xHC kernel must move per launch.  xhc_route reads X once and
+    phi_read, writes x_in, H_pre, the scores, idx and w; xhc_conv_gs reads F_out
+    and the conv weights and writes V [T][r+1][C] fp32; xhc_sparse_update reads
+    V and the k routed rows of X, writes those rows back, reads phi_act and
+    writes the coefficients."""
+    R, Kr = 2 * N - m, r + 1
+    Pa = k * k + k * Kr
+    route = T * N * C * 2 + N * C * R * 2 + T * C * 2 + T * (N + (N - m) + 2 * k) * 4
+    conv = T * C * 2 + kappa_sum * C * 4 + T * Kr * C * 4
+    update = T * Kr * C * 4 + 2 * T * k * C * 2 + k * C * Pa * 2 + T * (2 * k + Pa) * 4
+    return {"xhc_route": route, "xhc_conv_gs": conv, "xhc_sparse_update": update}
+
+
+def mhc_bwd_bytes(T: int, n: int, C: int) -> int:
+    """Bytes the backward must move per call: X, F_out, dX_next and dx_in read once,
+    dX and dF_out written once, phi read and dphi written once (fp32)."""
+    P = n * n + 2 * n
+    return T * (n * C * 2 * 3 + C * 2 * 2) + n * C * P * (2 + 4)
+
+
+def run_secondary(args, local):
+    """Timing lines for the other kernels of the method (xHC sublayer, mHC backward)
+    on their own workloads; one JSON line, rank 0 of a single process."""
+    import torch
+    import synth
+    import stream_residual_connections_b200 as M
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+
+    def to_dev(a):
+        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16) \
+            if a.dtype == np.uint16 else torch.from_numpy(np.ascontiguousarray(a))
+        return t.to(device)
+
+    peak, peak_src = measured_peak()
+    K = args.steps
+    if args.workload == "xhc":
+        wl = dict(synth.WORKLOADS["xhc"])
+        if args.tokens:
+            wl["T"] = args.tokens
+        inp = synth.xhc_inputs(**wl)
+        T, N, k, m, C = inp["T"], inp["N"], inp["k"], inp["m"], inp["C"]
+        X = to_dev(inp["X"])
+        F = to_dev(inp["F"])
+        phi_read = to_dev(np.ascontiguousarray(inp["phi_read"].T))
+        b_read = to_dev(inp["b_read"])
+        conv_w = [to_dev(w) for w in inp["conv_w"]]
+        phi_act = to_dev(np.ascontiguousarray(inp["phi_act"].T))
+        b_act = to_dev(inp["b_act"])
+        r = len(inp["kappa"])
+        outs = dict(x_in=torch.empty((T, C), dtype=X.dtype, device=device),
+                    H_pre=torch.empty((T, N), device=device), score=torch.empty((T, N - m), device=device),
+                    idx=torch.empty((T, k), dtype=torch.int32, device=device),
+                    w=torch.empty((T, k), device=device))
+        V = torch.empty((T, r + 1, C), dtype=torch.float32, device=device)
+        Hr = torch.empty((T, k, k), device=device)
+        Hpo = torch.empty((T, k, r + 1), device=device)
+        names = ("xhc_route", "xhc_conv_gs", "xhc_sparse_update")
+
+        def launches():
+            yield lambda: M.xhc_route(X, phi_read, inp["alpha_read"], b_read, k, m, inp["eps"], stream=stream, **outs)
+            yield lambda: M.xhc_conv_gs(F, conv_w, V=V, stream=stream)
+            yield lambda: M.xhc_sparse_update(X, V, outs["idx"], outs["w"], phi_act, inp["alpha_act"], b_act,
+                                              inp["t_iters"], inp["eps"], H_res=Hr, H_post=Hpo, stream=stream)
+        nbytes = xhc_bytes(T, N, k, m, C, r, sum(inp["kappa"]))
+        desc = (f"xHC sublayer (xhc_route + xhc_conv_gs + xhc_sparse_update, X updated in place), T={T}, "
+                f"N={N}, k={k}, m={m}, C={C}, kappa={list(inp['kappa'])}, bf16 state, Sinkhorn 20 iterations")
+    else:
+        wl = dict(synth.WORKLOADS["mhc_bwd"])
+        if args.tokens:
+            wl["T"] = args.tokens
+        inp = synth.mhc_grad_inputs(**wl)
+        T, n, C = inp["T"], inp["n"], inp["C"]
+        X, F = to_dev(inp["X"]), to_dev(inp["F"])
+        phi = to_dev(np.ascontiguousarray(inp["phi"].T))
+        b = to_dev(inp["b"])
+        dXn, dxi = to_dev(inp["dX_next"]), to_dev(inp["dx_in"])
+        P = n * n + 2 * n
+        bufs = dict(dX=torch.empty_like(X), dF=torch.empty_like(F),
+                    dphi=torch.empty((P, n * C), device=device), dalpha=torch.empty(3, device=device),
+                    db=torch.empty(P, device=device),
+                    workspace=torch.empty(max(M.mhc_backward_workspace_bytes(T, n, C), 256), dtype=torch.uint8,
+                                          device=device))
+        names = ("mhc_backward",)
+
+        def launches():
+            yield lambda: M.mhc_backward(X, F, phi, inp["alpha"], b, dXn, dxi, 20, 1e-6, stream=stream, **bufs)
+        nbytes = {"mhc_backward": mhc_bwd_bytes(T, n, C)}
+        desc = f"mHC sublayer backward (recompute + unrolled Sinkhorn reverse), T={T}, n={n}, C={C}, bf16"
+
+    for _ in range(args.warmup):
+        for f in launches():
+            f()
+    torch.cuda.synchronize(device)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for kk in range(K):
+        ev[kk][0].record(stream)
+        for j, f in enumerate(launches()):
+            f()
+            ev[kk][j + 1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    ms = start.elapsed_time(end) / K
+    rows = {}
+    for j, name in enumerate(names):
+        kms = sum(e[j].elapsed_time(e[j + 1]) for e in ev) / K
+        gbs = nbytes[name] / (kms / 1e3) / 1e9
+        rows[name] = {"ms": kms, "algorithmic_bytes": nbytes[name], "achieved_gbs": gbs, "frac": gbs / peak}
+    print(json.dumps({"workload": args.workload, "config": desc, "steps": K, "warmup": args.warmup,
+                      "ms_per_step": ms, "tokens_per_s": T / (ms / 1e3), "kernels": rows, "peak_gbs": peak,
+                      "peak_source": peak_src}), flush=True)
+
+
 # ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the current
 # kernels on this workload (profiles/*.txt); None until captured for the
 # kernel version in the tree.
@@ -401,6 +520,8 @@ def main(argv=None):
     p.add_argument("--profile", action="store_true",
                    help="only warm-up + timed kernel launches (for ncu); no e2e, clocks or oracle")
     p.add_argument("--tokens", type=int, default=None, help="override T (profiling of small cases)")
+    p.add_argument("--workload", choices=("mhc_fwd", "xhc", "mhc_bwd"), default="mhc_fwd",
+                   help="mhc_fwd: the benchmark line; xhc / mhc_bwd: timing lines for the other kernels")
     args = p.parse_args(argv)
     if args.tokens:
         WORKLOAD["T"] = args.tokens
@@ -409,6 +530,9 @@ def main(argv=None):
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args, world, rank)
+        return 0
+    if args.workload != "mhc_fwd":
+        run_secondary(args, local)
         return 0
     run_ours(args, world, rank, local)
     return 0

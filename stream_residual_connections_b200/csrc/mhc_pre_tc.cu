@@ -36,8 +36,7 @@
 //          the receivers' mbarriers, so no fence or remote arrive sits on this
 //          path.
 //   2-3, 8-15  x_in = H_pre X for this CTA's channels, re-reading the tile's
-//          X slice from L2 (evict-first on this last read); the epilogue
-//          warps join them once the tile's H_pre has landed.
+//          X slice from L2 (evict-first on this last read).
 // The roles meet only through mbarriers and one progress counter, so the TMA
 // ring keeps streaming while a tile's coefficients and x_in are produced.
 //
@@ -54,22 +53,29 @@ namespace pretc {
 
 using namespace sm100;
 
+constexpr int CL = 8;            // CTAs per cluster (channel split)
 constexpr int MROWS = 128;       // MMA M (TMEM lanes): two streams of up to MT_CAP tokens
 constexpr int MT_CAP = 64;       // token rows per tile: bounds the L2 footprint of the x_in re-read
 constexpr int KC = 64;           // channels per block (one 128-byte row)
 constexpr int MAX_STAGES = 6;
 constexpr int SMEM_LIMIT = 227 * 1024;
 constexpr int NTHREADS = 512;
-constexpr int COEF_WARP0 = 2;                                     // warps 2-3: coefficients
-constexpr int EPI_WARP0 = 4, EPI_WARPS = 4;                       // warps 4-7: TMEM lane quarters 0-3
-constexpr int XIN_WARP0 = 8, XIN_WARPS = 8, XIN_THREADS = XIN_WARPS * 32;   // warps 8-15
+constexpr int EPI_WARP0 = 4, EPI_WARPS = 4;                       // TMEM lane quarters 0-3
+constexpr int XIN_WARPS = 10, XIN_THREADS = XIN_WARPS * 32;       // warps 2-3 and 8-15
+constexpr int TOK_PER_CTA = MT_CAP / CL;  // tokens whose coefficients a CTA computes
 constexpr int XIN_UNROLL = 4;             // x_in vectors in flight per thread
-// L2 bytes that the tiles loaded but not yet re-read by x_in may occupy
-#ifndef MHC_PRE_L2_BUDGET_MB
-#define MHC_PRE_L2_BUDGET_MB 96
+// Tiles the TMA stream may run ahead of x_in.  With 15 clusters of 64-token
+// tiles, LAG + 1 tiles of X (about 31 MB each at n = 4, C = 4096) wait in L2
+// for their re-read: at LAG = 3 part of the re-read already misses L2 (about
+// 60 of 256 MB, measured), yet the kernel is faster than at LAG = 2, where
+// the ring idles while x_in catches up.
+#ifndef MHC_PRE_LAG
+#define MHC_PRE_LAG 3
 #endif
+constexpr int LAG = MHC_PRE_LAG;
 constexpr int ACC_COLS = 256;             // TMEM columns per accumulator buffer
 constexpr int TMEM_COLS = 512;
+static_assert(TOK_PER_CTA * 8 == 64, "warps 4-5: one 8-lane group per coefficient token");
 
 template <int N> struct Cfg {
     static constexpr int P = N * N + 2 * N;
@@ -84,39 +90,35 @@ template <int N> struct Cfg {
 };
 
 enum Bar { B_FULL = 0, B_EMPTY = B_FULL + MAX_STAGES, B_TFULL = B_EMPTY + MAX_STAGES, B_TEMPTY = B_TFULL + 2,
-           B_PART = B_TEMPTY + 2, B_HPRE = B_PART + 2, B_XIN = B_HPRE + 2, B_DRAIN, B_COUNT };
+           B_PART = B_TEMPTY + 2, B_HPRE, B_XIN = B_HPRE + 2, B_DRAIN, B_COUNT };
 
 struct Layout {
     uint32_t ring, part, hpre, bias, bars, slot, total;
     int stages;
 };
 
-// Bytes after the ring: partial rows [2 tiles][cluster CTA][2 halves][token of
-// the owner][PSP] (cluster size x tokens per CTA = MT_CAP), H_pre
+// Bytes after the ring: partial rows [CL][2 halves][TOK_PER_CTA][PSP], H_pre
 // [2][MT_CAP][N], b, barriers.
 template <int N>
 __host__ __device__ constexpr uint32_t layout_fixed_bytes() {
     using G = Cfg<N>;
-    return 2 * 2 * MT_CAP * G::PSP * 4 + 2 * MT_CAP * N * 4 + G::P * 4 + 16 + B_COUNT * 8 + 16;
+    return CL * 2 * TOK_PER_CTA * G::PSP * 4 + 2 * MT_CAP * N * 4 + G::P * 4 + 16 + B_COUNT * 8 + 16;
 }
 
-// Ring stages that fit next to the fixed part of the 227 KB.
+// Shared memory plan: the ring takes as many stages (up to MAX_STAGES) as the
+// rest of the 227 KB leaves room for.
 template <int N>
-__host__ __device__ constexpr int stages_fit() {
-    constexpr int64_t room = int64_t(SMEM_LIMIT) - 1024 - layout_fixed_bytes<N>();
-    constexpr int64_t fit = room > 0 ? room / Cfg<N>::STAGE_BYTES : 0;
-    return int(fit < MAX_STAGES ? fit : MAX_STAGES);
-}
-
-// Shared memory plan for a ring of `stages` stages.
-template <int N>
-__host__ __device__ inline Layout layout_for(int stages) {
+__host__ __device__ inline Layout layout_for() {
     using G = Cfg<N>;
     Layout L;
     L.ring = 0;
-    L.stages = stages;
+    {
+        const int64_t room = int64_t(SMEM_LIMIT) - 1024 - layout_fixed_bytes<N>();
+        const int64_t fit = room > 0 ? room / G::STAGE_BYTES : 0;
+        L.stages = int(fit < MAX_STAGES ? fit : MAX_STAGES);
+    }
     L.part = L.ring + uint32_t(L.stages) * G::STAGE_BYTES;
-    L.hpre = L.part + 2 * 2 * MT_CAP * G::PSP * 4;
+    L.hpre = L.part + CL * 2 * TOK_PER_CTA * G::PSP * 4;
     L.bias = L.hpre + 2 * MT_CAP * N * 4;
     L.bars = (L.bias + G::P * 4 + 15) / 16 * 16;
     L.slot = L.bars + B_COUNT * 8;
@@ -138,60 +140,11 @@ __device__ __forceinline__ void row_slot(int r, int Mt, int& h, int& tok) {
     }
 }
 
-// x_in rows [t0, t0 + rows) of this CTA's channels [c0, c0 + Cs): thread xt of
-// nthr takes 16-byte vectors xt, xt + nthr, ... (XIN_UNROLL of them in flight).
 template <int N>
-__device__ __forceinline__ void xin_tile(const bf16_t* __restrict__ X, bf16_t* __restrict__ x_in,
-                                         const float* hb, int64_t t0, int rows, int C, int c0, int Cs,
-                                         int xt, int nthr, uint64_t drop)
-{
-    const int VPT = Cs / 8;                          // 16-byte vectors per token
-    const int items = rows * VPT;
-    for (int w0 = xt; w0 < items; w0 += XIN_UNROLL * nthr) {
-        uint4 raw[XIN_UNROLL][N];
-        int tk[XIN_UNROLL], cc[XIN_UNROLL];
-#pragma unroll
-        for (int u = 0; u < XIN_UNROLL; ++u) {
-            const int w = w0 + u * nthr;
-            const int wc = w < items ? w : items - 1;   // clamp; the store is skipped
-            tk[u] = wc / VPT;
-            cc[u] = c0 + (wc - tk[u] * VPT) * 8;
-#pragma unroll
-            for (int i = 0; i < N; ++i)
-                raw[u][i] = ldg16_raw_hint(X + ((t0 + tk[u]) * N + i) * C + cc[u], drop);
-        }
-#pragma unroll
-        for (int u = 0; u < XIN_UNROLL; ++u) {
-            if (w0 + u * nthr >= items) break;
-            float o[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) o[e] = 0.0f;
-#pragma unroll
-            for (int i = 0; i < N; ++i) {
-                const float hh = hb[tk[u] * N + i];
-                const uint32_t w4[4] = {raw[u][i].x, raw[u][i].y, raw[u][i].z, raw[u][i].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    o[2 * e] = fmaf(hh, bf16_lo(w4[e]), o[2 * e]);
-                    o[2 * e + 1] = fmaf(hh, bf16_hi(w4[e]), o[2 * e + 1]);
-                }
-            }
-            store16<false>(x_in + (t0 + tk[u]) * C + cc[u], o);
-        }
-    }
-}
-
-// Launched in clusters of CL CTAs (8, or 16 where C allows; the cluster size
-// is a launch attribute).  stages: ring depth; phi_resident: the ring is a
-// multiple of the channel blocks per tile, slot s always holds block s mod CB,
-// and its phiT rows, loaded on the slot's first use, stay; lag: tiles the TMA
-// stream may run ahead of x_in.
-template <int N, int CL>
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NTHREADS, 1)
 pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmPhi,
               const bf16_t* __restrict__ X, float a0, float a1, float a2,
-              const float* __restrict__ b, int64_t T, int C, int Mt, int num_tiles, int stages,
-              int phi_resident, int lag, int t_iters,
+              const float* __restrict__ b, int64_t T, int C, int Mt, int num_tiles, int t_iters,
               float eps, bf16_t* __restrict__ x_in, float* __restrict__ Hpre,
               float* __restrict__ Hpost, float* __restrict__ Hres, float* __restrict__ u_out,
               float* __restrict__ r_out)
@@ -199,18 +152,16 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     using G = Cfg<N>;
     constexpr int P = G::P, R = G::R, NP = G::NP, PS = G::PS, PSP = G::PSP;
     constexpr int STAGE_BYTES = G::STAGE_BYTES, PAIR_BYTES = G::PAIR_BYTES;
-    constexpr int TOK_PER_CTA = MT_CAP / CL;       // tokens whose coefficients a CTA computes
-    static_assert(TOK_PER_CTA * CL == 64, "warps 4-5: one CL-lane group per coefficient token");
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte-swizzle atoms
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int Cs = C / CL;
     const int CB = Cs / KC;            // channel blocks = ring stages per tile
-    const Layout L = layout_for<N>(stages);
+    const Layout L = layout_for<N>();
     const int STAGES = L.stages;
     uint8_t* sring = smem + L.ring;
-    float* rpart = reinterpret_cast<float*>(smem + L.part);   // [2][CL][2][TOK_PER_CTA][PSP], pushed by the cluster
+    float* rpart = reinterpret_cast<float*>(smem + L.part);   // [CL][2][TOK_PER_CTA][PSP], pushed by the cluster
     float* shpre = reinterpret_cast<float*>(smem + L.hpre);   // [2][MT_CAP][N]
     float* sb = reinterpret_cast<float*>(smem + L.bias);      // b, kept on chip for the coefficients
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
@@ -218,7 +169,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
     uint64_t* empty = bars + B_EMPTY;
     uint64_t* tfull = bars + B_TFULL;
     uint64_t* tempty = bars + B_TEMPTY;
-    uint64_t* part_full = bars + B_PART;     // [2] this CTA's tokens: all partial rows of a tile landed
+    uint64_t* part_full = bars + B_PART;     // this CTA's tokens: all partial rows landed
     uint64_t* hpre_full = bars + B_HPRE;     // [2] H_pre of every tile row landed (per tile parity)
     uint64_t* xin_prog = bars + B_XIN;
     uint64_t* drain = bars + B_DRAIN;
@@ -245,8 +196,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         }
         // one local arrival (with the expected byte count) per phase; the bytes
         // come from st.async pushes of the cluster
-        mbar_init(&part_full[0], 1);
-        mbar_init(&part_full[1], 1);
+        mbar_init(part_full, 1);
         mbar_init(&hpre_full[0], 1);
         mbar_init(&hpre_full[1], 1);
         mbar_init(xin_prog, XIN_WARPS);
@@ -268,7 +218,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             const uint64_t keep = policy_evict_last();
-            const uint32_t x_tx = uint32_t(NP) * uint32_t(2 * Mt) * 128, phi_tx = uint32_t(NP) * uint32_t(2 * R) * 128;
+            const uint32_t stage_tx = uint32_t(NP) * uint32_t(2 * R + 2 * Mt) * 128;
             int s = 0;
             uint32_t ph = 0;
             int inflight_s[MAX_STAGES], inflight_ph[MAX_STAGES], n_issued = 0;
@@ -277,8 +227,8 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             for (int tile = cluster_id; tile < num_tiles && ok; tile += nclusters, ++it) {
                 const int t0 = tile * Mt;
                 // keep the re-read of tile it-LAG in L2: do not run further ahead of x_in
-                if (it >= lag) {
-                    const int need = XIN_WARPS * (it - lag + 1);
+                if (it >= LAG) {
+                    const int need = XIN_WARPS * (it - LAG + 1);
                     long long k = 0;
                     while (*(volatile int*)&s_xin_done < need && !*(volatile int*)&s_abort && k < g_wait_limit) {
                         __nanosleep(64);
@@ -288,14 +238,13 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                 }
                 for (int cb = 0; cb < CB; ++cb) {
                     if (!mbar_wait(&empty[s], ph ^ 1) || *(volatile int*)&s_abort) { ok = false; break; }
-                    const bool with_phi = !phi_resident || n_issued < STAGES;
-                    mbar_arrive_expect_tx(&full[s], x_tx + (with_phi ? phi_tx : 0u));
+                    mbar_arrive_expect_tx(&full[s], stage_tx);
                     const int cc = c0 + cb * KC;
 #pragma unroll
                     for (int p = 0; p < NP; ++p) {
                         uint8_t* pb = sring + s * STAGE_BYTES + p * PAIR_BYTES;
                         // phiT {64 channels, R rows, streams 2p..2p+1} of the {C, P, n} view
-                        if (with_phi) tma_load_3d_hint(pb, &tmPhi, &full[s], cc, 0, 2 * p, keep);
+                        tma_load_3d_hint(pb, &tmPhi, &full[s], cc, 0, 2 * p, keep);
                         // X {64 channels, Mt tokens, streams 2p..2p+1} of the {C, T, n} view
                         tma_load_3d_hint(pb + 2 * R * 128, &tmX, &full[s], cc, t0, 2 * p, keep);
                     }
@@ -355,10 +304,13 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         }
 
     } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + EPI_WARPS) {
-        // ------------------------------------------------------------ TMEM -> owners
+        // ------------------------------------------------------------ epilogue
+        const int et = threadIdx.x - EPI_WARP0 * 32;    // 0..127
         const int qd = warp & 3;                        // TMEM lane quarter of this warp
         const int r = qd * 32 + lane;                   // TMEM row (lane)
-        constexpr int PART_FLOATS = CL * 2 * TOK_PER_CTA * PSP;
+        const float inv_K = 1.0f / float(N * C);
+        constexpr uint32_t PART_BYTES = CL * 2 * TOK_PER_CTA * PSP * 4;
+        constexpr uint32_t HPRE_BYTES = MT_CAP * N * 4;
         int h, tok;
         row_slot(r, Mt, h, tok);
         // the partial row goes to the token's owner CTA, slot (rank, half, token % TOK_PER_CTA)
@@ -368,8 +320,15 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
         const uint32_t push_bar = mapa(smem_u32(part_full), owner);
         int it = 0;
         for (int tile = cluster_id; tile < num_tiles; tile += nclusters, ++it) {
+            const int64_t t0 = int64_t(tile) * Mt;
             const int acc = it & 1;
-            if (!warp_wait(&tfull[acc], uint32_t((it >> 1) & 1))) { s_abort = 1; break; }
+            const uint32_t par = uint32_t((it >> 1) & 1);
+            if (et == 0) {
+                // expected bytes of this tile's phases; pushes may land before or after
+                mbar_arrive_expect_tx(part_full, PART_BYTES);
+                mbar_arrive_expect_tx(&hpre_full[acc], HPRE_BYTES);
+            }
+            if (!warp_wait(&tfull[acc], par)) { s_abort = 1; break; }
             tc_fence_after();
             float d[2 * R];
             const uint32_t taddr = tmem_base + (uint32_t(qd * 32) << 16) + uint32_t(acc * ACC_COLS);
@@ -397,12 +356,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             // H_pre of tile it lands in buffer it&1, last read by the x_in warps for
             // tile it-2: they must have moved on (they arrive after their tile it-1 wait)
             if (it >= 1 && !warp_wait(xin_prog, uint32_t((it - 1) & 1))) { s_abort = 1; break; }
-            // partial-row buffer it&1 of every owner was last read for tile it-2; the
-            // owners are done with it once this CTA holds H_pre of tile it-2
-            if (it >= 2 && !warp_wait(&hpre_full[acc], uint32_t(((it - 2) >> 1) & 1))) { s_abort = 1; break; }
             // push (partial projections, sum of squares) of this row's half to its owner
-            const uint32_t dst = push_dst + uint32_t(acc * PART_FLOATS * 4);
-            const uint32_t bar = push_bar + uint32_t(acc * 8);
 #pragma unroll
             for (int p = 0; p < PSP; p += 4) {
                 float w[4];
@@ -411,116 +365,129 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
                     const int q = p + e;
                     w[e] = q < P ? (h ? d[R + q] : d[q]) : (q == P ? ss : 0.0f);   // q < P <= R
                 }
-                st_async_f32x4(dst + p * 4, make_float4(w[0], w[1], w[2], w[3]), bar);
+                st_async_f32x4(push_dst + p * 4, make_float4(w[0], w[1], w[2], w[3]), push_bar);
             }
-        }
-    } else if (warp >= COEF_WARP0 && warp < COEF_WARP0 + 2) {
-        // ------------------------------------------------------------ coefficients
-        // This CTA's TOK_PER_CTA tokens of every tile: a group of CL lanes per
-        // token.  Lane g sums entries p = g (mod CL) over the 2 x CL partial rows,
-        // then the group exchanges the sums (independent shuffles, no reduction
-        // chain); lane g < N carries row g of H_res.
-        const int et = threadIdx.x - COEF_WARP0 * 32;   // 0..63
-        const float inv_K = 1.0f / float(N * C);
-        constexpr uint32_t PART_BYTES = CL * 2 * TOK_PER_CTA * PSP * 4;
-        constexpr uint32_t HPRE_BYTES = MT_CAP * N * 4;
-        constexpr int PART_FLOATS = CL * 2 * TOK_PER_CTA * PSP;
-        const int jj = et / CL, g = et % CL;
-        int it = 0;
-        for (int tile = cluster_id; tile < num_tiles; tile += nclusters, ++it) {
-            const int64_t t0 = int64_t(tile) * Mt;
-            const int bb = it & 1;
-            bool ok = true;
-            if (et == 0) {
-                // re-arm this tile's receive barriers once their previous phases (tile
-                // it-2) are over; pushes of this tile may land before or after
-                if (it >= 2 && !mbar_wait(&hpre_full[bb], uint32_t(((it - 2) >> 1) & 1))) ok = false;
-                mbar_arrive_expect_tx(&part_full[bb], PART_BYTES);
-                mbar_arrive_expect_tx(&hpre_full[bb], HPRE_BYTES);
-            }
-            ok = ok && mbar_wait(&part_full[bb], uint32_t((it >> 1) & 1)) && !*(volatile int*)&s_abort;
-            if (!__all_sync(0xffffffffu, ok)) {
-                s_abort = 1;
-                break;
-            }
-            const float* part = rpart + bb * PART_FLOATS;
-            const int j = int(rank) * TOK_PER_CTA + jj;     // row within the tile
-            constexpr int OWN = (PS + CL - 1) / CL;         // entries summed per lane
-            float own[OWN];
+            if (et < 64) {
+                if (!warp_wait(part_full, uint32_t(it & 1))) { s_abort = 1; break; }
+                // Coefficients of this CTA's TOK_PER_CTA tokens: a group of 8 lanes per
+                // token.  Lane g sums entries p = g (mod 8) over the 2 x CL partial
+                // rows, then the group exchanges the sums (independent shuffles, no
+                // reduction chain); lane g < N later carries row g of H_res.
+                const int jj = et >> 3, g = et & 7;
+                const int j = int(rank) * TOK_PER_CTA + jj;     // row within the tile
+                constexpr int OWN = (PS + 7) / 8;               // entries summed per lane
+                float own[OWN];
 #pragma unroll
-            for (int k = 0; k < OWN; ++k) {
-                const int p = g + CL * k;
-                float s0 = 0.0f, s1 = 0.0f;
-                if (p < PS) {
+                for (int k = 0; k < OWN; ++k) {
+                    const int p = g + 8 * k;
+                    float s0 = 0.0f, s1 = 0.0f;
+                    if (p < PS) {
 #pragma unroll
-                    for (int c = 0; c < CL; ++c) {
-                        s0 += part[((c * 2 + 0) * TOK_PER_CTA + jj) * PSP + p];
-                        s1 += part[((c * 2 + 1) * TOK_PER_CTA + jj) * PSP + p];
+                        for (int c = 0; c < CL; ++c) {
+                            s0 += rpart[((c * 2 + 0) * TOK_PER_CTA + jj) * PSP + p];
+                            s1 += rpart[((c * 2 + 1) * TOK_PER_CTA + jj) * PSP + p];
+                        }
+                    }
+                    own[k] = s0 + s1;
+                }
+                float v[PSP];
+#pragma unroll
+                for (int p = 0; p < PS; ++p) v[p] = __shfl_sync(0xffffffffu, own[p >> 3], p & 7, 8);
+                const float rr_ = sqrtf(v[P] * inv_K + eps);                   // Eq.(15)
+                const float inv_r = 1.0f / rr_;
+                // every lane of the group carries the whole n x n Sinkhorn (no shuffles in
+                // the iterations); lane g < N then keeps stream g's gates and H_res row g
+                float mres[N][N];
+#pragma unroll
+                for (int i = 0; i < N; ++i)
+#pragma unroll
+                    for (int k = 0; k < N; ++k)
+                        mres[i][k] = a2 * v[2 * N + i * N + k] * inv_r + sb[2 * N + i * N + k];   // Eq.(16)
+                sinkhorn_regs<N>(mres, t_iters);                                   // Eq.(19)
+                float zpre = 0.0f, zpost = 0.0f, row[N];
+#pragma unroll
+                for (int k = 0; k < N; ++k) row[k] = 0.0f;
+#pragma unroll
+                for (int i = 0; i < N; ++i)
+                    if (g == i) {
+                        zpre = a0 * v[i] * inv_r + sb[i];
+                        zpost = a1 * v[N + i] * inv_r + sb[N + i];
+#pragma unroll
+                        for (int k = 0; k < N; ++k) row[k] = mres[i][k];
+                    }
+                if (g < N) {
+                    const float hp = sigmoidf_(zpre);                              // Eq.(17)
+                    // every CTA needs H_pre of every tile row for its x_in channels
+                    const uint32_t hoff = smem_u32(shpre + (acc * MT_CAP + j) * N + g);
+                    const uint32_t hbar = smem_u32(&hpre_full[acc]);
+                    for (uint32_t cr = 0; cr < CL; ++cr) st_async_f32(mapa(hoff, cr), hp, mapa(hbar, cr));
+                    const int64_t t = t0 + j;
+                    if (j < Mt && t < T) {
+                        if (Hpost) Hpost[t * N + g] = 2.0f * sigmoidf_(zpost);     // Eq.(18)
+                        if (Hpre) Hpre[t * N + g] = hp;
+                        if (Hres) {
+#pragma unroll
+                            for (int k = 0; k < N; ++k) Hres[(t * N + g) * N + k] = row[k];
+                        }
                     }
                 }
-                own[k] = s0 + s1;
-            }
-            float v[PSP];
+                if (u_out && j < Mt && t0 + j < T) {       // the backward's recompute
 #pragma unroll
-            for (int p = 0; p < PS; ++p) v[p] = __shfl_sync(0xffffffffu, own[p / CL], p % CL, CL);
-            const float rr_ = sqrtf(v[P] * inv_K + eps);                   // Eq.(15)
-            const float inv_r = 1.0f / rr_;
-            // every lane of the group carries the whole n x n Sinkhorn (no shuffles in
-            // the iterations); lane g < N then keeps stream g's gates and H_res row g
-            float mres[N][N];
-#pragma unroll
-            for (int i = 0; i < N; ++i)
-#pragma unroll
-                for (int k = 0; k < N; ++k)
-                    mres[i][k] = a2 * v[2 * N + i * N + k] * inv_r + sb[2 * N + i * N + k];   // Eq.(16)
-            sinkhorn_regs<N>(mres, t_iters);                                   // Eq.(19)
-            float zpre = 0.0f, zpost = 0.0f, row[N];
-#pragma unroll
-            for (int k = 0; k < N; ++k) row[k] = 0.0f;
-#pragma unroll
-            for (int i = 0; i < N; ++i)
-                if (g == i) {
-                    zpre = a0 * v[i] * inv_r + sb[i];
-                    zpost = a1 * v[N + i] * inv_r + sb[N + i];
-#pragma unroll
-                    for (int k = 0; k < N; ++k) row[k] = mres[i][k];
-                }
-            if (g < N) {
-                const float hp = sigmoidf_(zpre);                              // Eq.(17)
-                // every CTA needs H_pre of every tile row for its x_in channels
-                const uint32_t hoff = smem_u32(shpre + (bb * MT_CAP + j) * N + g);
-                const uint32_t hbar = smem_u32(&hpre_full[bb]);
-                for (uint32_t cr = 0; cr < CL; ++cr) st_async_f32(mapa(hoff, cr), hp, mapa(hbar, cr));
-                const int64_t t = t0 + j;
-                if (j < Mt && t < T) {
-                    if (Hpost) Hpost[t * N + g] = 2.0f * sigmoidf_(zpost);     // Eq.(18)
-                    if (Hpre) Hpre[t * N + g] = hp;
-                    if (Hres) {
-#pragma unroll
-                        for (int k = 0; k < N; ++k) Hres[(t * N + g) * N + k] = row[k];
-                    }
+                    for (int p = 0; p < P; ++p)
+                        if ((p & 7) == g) u_out[(t0 + j) * P + p] = v[p] * inv_r;
+                    if (g == 0) r_out[t0 + j] = rr_;
                 }
             }
-            if (u_out && j < Mt && t0 + j < T) {       // the backward's recompute
-#pragma unroll
-                for (int p = 0; p < P; ++p)
-                    if (p % CL == g) u_out[(t0 + j) * P + p] = v[p] * inv_r;
-                if (g == 0) r_out[t0 + j] = rr_;
-            }
+            // every owner has read its partial rows of this tile once this CTA holds the
+            // tile's H_pre; only then may the next tile's partial rows be pushed
+            if (!warp_wait(&hpre_full[acc], par)) { s_abort = 1; break; }
         }
-    } else if (warp >= XIN_WARP0) {
+    } else {
         // ------------------------------------------------------------ x_in
-        const int xt = (warp - XIN_WARP0) * 32 + lane;
+        const int xt = (warp < EPI_WARP0 ? warp - 2 : warp - (EPI_WARP0 + EPI_WARPS - 2)) * 32 + lane;
         const uint64_t drop = policy_evict_first();
+        const int VPT = Cs / 8;                          // 16-byte vectors per token
         int it = 0;
         for (int tile = cluster_id; tile < num_tiles; tile += nclusters, ++it) {
             if (!warp_wait_sleep(&hpre_full[it & 1], uint32_t((it >> 1) & 1))) { s_abort = 1; break; }
             __syncwarp();
             if (lane == 0) mbar_arrive(xin_prog);
             const int64_t t0 = int64_t(tile) * Mt;
+            const float* hb = shpre + (it & 1) * MT_CAP * N;
             const int rows = int((T - t0) < int64_t(Mt) ? (T - t0) : int64_t(Mt));
-            if (x_in)
-                xin_tile<N>(X, x_in, shpre + (it & 1) * MT_CAP * N, t0, rows, C, c0, Cs, xt, XIN_THREADS, drop);
+            const int items = x_in ? rows * VPT : 0;
+            for (int w0 = xt; w0 < items; w0 += XIN_UNROLL * XIN_THREADS) {
+                uint4 raw[XIN_UNROLL][N];
+                int tk[XIN_UNROLL], cc[XIN_UNROLL];
+#pragma unroll
+                for (int u = 0; u < XIN_UNROLL; ++u) {
+                    const int w = w0 + u * XIN_THREADS;
+                    const int wc = w < items ? w : items - 1;   // clamp; the store is skipped
+                    tk[u] = wc / VPT;
+                    cc[u] = c0 + (wc - tk[u] * VPT) * 8;
+#pragma unroll
+                    for (int i = 0; i < N; ++i)
+                        raw[u][i] = ldg16_raw_hint(X + ((t0 + tk[u]) * N + i) * C + cc[u], drop);
+                }
+#pragma unroll
+                for (int u = 0; u < XIN_UNROLL; ++u) {
+                    if (w0 + u * XIN_THREADS >= items) break;
+                    float o[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) o[e] = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < N; ++i) {
+                        const float hh = hb[tk[u] * N + i];
+                        const uint32_t w4[4] = {raw[u][i].x, raw[u][i].y, raw[u][i].z, raw[u][i].w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            o[2 * e] = fmaf(hh, bf16_lo(w4[e]), o[2 * e]);
+                            o[2 * e + 1] = fmaf(hh, bf16_hi(w4[e]), o[2 * e + 1]);
+                        }
+                    }
+                    store16<false>(x_in + (t0 + tk[u]) * C + cc[u], o);
+                }
+            }
             __syncwarp();
             if (lane == 0) atomicAdd(&s_xin_done, 1);
         }
@@ -555,52 +522,42 @@ static EncodeTiledFn encode_fn()
 }
 
 template <int N>
-static int smem_bytes(int stages) { return int(layout_for<N>(stages).total) + 1024; }
+static int smem_bytes() { return int(layout_for<N>().total) + 1024; }
 
 template <int N>
 static bool fits(int C)
 {
-    return C % (8 * KC) == 0 && stages_fit<N>() >= 2 && smem_bytes<N>(stages_fit<N>()) <= SMEM_LIMIT;
+    return C % (CL * KC) == 0 && layout_for<N>().stages >= 2 && smem_bytes<N>() <= SMEM_LIMIT;
 }
 
-// Clusters of CL CTAs that can be resident at once (0 if none), per kernel.
-template <int N, int CL>
-static int max_active_clusters()
+template <int N>
+static mhc_status launch_n(const PreArgs& a, cudaStream_t s)
 {
-    static int cached = -1;
-    if (cached >= 0) return cached;
-    auto kern = pre_tc_kernel<N, CL>;
-    const int smem = smem_bytes<N>(stages_fit<N>());
-    cached = 0;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 0;
-    if (CL > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-        return 0;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(CL * 64);
-    cfg.blockDim = dim3(NTHREADS);
-    cfg.dynamicSmemBytes = size_t(smem);
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = CL; attr.val.clusterDim.y = 1; attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr; cfg.numAttrs = 1;
-    int nc = 0;
-    if (cudaOccupancyMaxActiveClusters(&nc, kern, &cfg) != cudaSuccess) { (void)cudaGetLastError(); nc = 0; }
-    cached = nc > 0 ? nc : 0;
-    return cached;
-}
-
-template <int N, int CL>
-static mhc_status launch_cl(const PreArgs& a, int max_clusters, cudaStream_t s)
-{
-    auto kern = pre_tc_kernel<N, CL>;
-    // Ring: in phi-resident mode a multiple of the CB channel blocks per tile
-    // (slot s always holds block s mod CB); otherwise as deep as fits.
-    const int fit = stages_fit<N>();
-    const int CB = a.C / CL / KC;
-    const bool resident = CB <= fit;
-    const int stages = resident ? (fit / CB) * CB : fit;
-    const int smem = smem_bytes<N>(stages);
-
+    static int configured_smem = 0;
+    static int max_clusters = 0;
+    const int smem = smem_bytes<N>();
+    auto kern = pre_tc_kernel<N>;
+    if (smem > configured_smem) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return cuda_status(e, "mhc_pre (tc): set shared memory size");
+        configured_smem = smem;
+        max_clusters = 0;
+    }
+    if (max_clusters == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(CL * 64);
+        cfg.blockDim = dim3(NTHREADS);
+        cfg.dynamicSmemBytes = size_t(configured_smem);
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = CL; attr.val.clusterDim.y = 1; attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr; cfg.numAttrs = 1;
+        int nc = 0;
+        cudaError_t e = cudaOccupancyMaxActiveClusters(&nc, kern, &cfg);
+        if (e != cudaSuccess || nc <= 0) return cuda_status(e != cudaSuccess ? e : cudaErrorInvalidConfiguration,
+                                                             "mhc_pre (tc): cluster occupancy");
+        max_clusters = nc;
+    }
     // Token tiles of Mt rows, Mt a multiple of 8 (each stream's rows in a stage
     // then start on a 1024-byte swizzle atom) and at most MT_CAP.  A tile costs
     // its Mt tokens plus a fixed overhead worth about TILE_COST tokens (the MMAs
@@ -616,11 +573,6 @@ static mhc_status launch_cl(const PreArgs& a, int max_clusters, cudaStream_t s)
     }
     const int64_t tiles64 = (a.T + Mt - 1) / Mt;
     const int nclusters = int(tiles64 < max_clusters ? tiles64 : max_clusters);
-    // How far the TMA stream may run ahead of x_in: the tiles loaded but not yet
-    // re-read (lag + 1 per cluster) must stay within the L2 budget.
-    const double step_bytes = double(nclusters) * Mt * a.n * double(a.C) * 2.0;
-    int lag = int(double(MHC_PRE_L2_BUDGET_MB) * 1048576.0 / step_bytes) - 1;
-    lag = lag < 1 ? 1 : (lag > 6 ? 6 : lag);
 
     EncodeTiledFn enc = encode_fn();
     if (!enc) {
@@ -659,40 +611,11 @@ static mhc_status launch_cl(const PreArgs& a, int max_clusters, cudaStream_t s)
             return MHC_ERR_CUDA;
         }
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(unsigned(nclusters * CL));
-    cfg.blockDim = dim3(NTHREADS);
-    cfg.dynamicSmemBytes = size_t(smem);
-    cfg.stream = s;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = CL; attr.val.clusterDim.y = 1; attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr; cfg.numAttrs = 1;
-    const bf16_t* Xp = static_cast<const bf16_t*>(a.X);
-    bf16_t* xin = a.skip_xin ? nullptr : static_cast<bf16_t*>(a.x_in);
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mapX, mapPhi, Xp, a.alpha[0], a.alpha[1], a.alpha[2], a.b,
-                                             a.T, a.C, Mt, int(tiles64), stages, int(resident), lag, a.t_iters,
-                                             a.eps, xin, a.H_pre, a.H_post, a.H_res, a.u_out, a.r_out);
-    if (e != cudaSuccess) return cuda_status(e, "mhc_pre (tc) kernel launch");
+    kern<<<dim3(unsigned(nclusters * CL)), NTHREADS, size_t(smem), s>>>(
+        mapX, mapPhi, static_cast<const bf16_t*>(a.X), a.alpha[0], a.alpha[1], a.alpha[2], a.b, a.T,
+        a.C, Mt, int(tiles64), a.t_iters, a.eps, a.skip_xin ? nullptr : static_cast<bf16_t*>(a.x_in),
+        a.H_pre, a.H_post, a.H_res, a.u_out, a.r_out);
     return launch_status("mhc_pre (tc) kernel");
-}
-
-// Clusters of 16 CTAs when C splits into 16 slices of whole channel blocks
-// (each CTA then holds a quarter of the phiT rows it would hold in a cluster of
-// 8, which leaves room to keep them resident), else clusters of 8.
-template <int N>
-static mhc_status launch_n(const PreArgs& a, cudaStream_t s)
-{
-    if (a.C % (16 * KC) == 0) {
-        const int nc = max_active_clusters<N, 16>();
-        if (nc > 0) return launch_cl<N, 16>(a, nc, s);
-    }
-    const int nc = max_active_clusters<N, 8>();
-    if (nc <= 0) {
-        set_error("mhc_pre (tc): no cluster of 8 CTAs fits on this device");
-        return MHC_ERR_CUDA;
-    }
-    return launch_cl<N, 8>(a, nc, s);
 }
 
 }  // namespace pretc

@@ -170,10 +170,9 @@ def restore_path():
                                    (700, 4, 7168), (333, 3, 7168), (901, 4, 1536), (450, 2, 3072),
                                    (5000, 4, 4096)])
 def test_tensor_core_path_shapes(T, n, C, restore_path):
-    """TMA + tcgen05 projection: one and several tiles per cluster, ragged last
-    tile, n = 2, 3, 4; clusters of 8 CTAs (C = 512, 1536) and of 16 (C a
-    multiple of 1024); phiT resident in the ring (up to 4 channel blocks per
-    CTA) or streamed with X (C = 7168: 7 blocks per CTA)."""
+    """TMA + tcgen05 projection (8-CTA clusters): one and several tiles per
+    cluster, ragged last tile (Mt from 8 to 64 rows), n = 2, 3 (a zero-filled
+    fourth stream), 4; one to 14 channel blocks per CTA (C = 512 ... 7168)."""
     M.mhc_set_path(M.MHC_PATH_TENSOR)
     inp = synth.mhc_inputs(T, n, C, "bf16", seed=400 + T + n + C)
     _compare(inp, _run(inp))
