@@ -431,7 +431,8 @@ def run_secondary(args, local):
         F = to_dev(inp["F"])
         phi_read = to_dev(np.ascontiguousarray(inp["phi_read"].T))
         b_read = to_dev(inp["b_read"])
-        conv_w = [to_dev(w) for w in inp["conv_w"]]
+        kappa = [int(x) for x in inp["kappa"]]
+        conv_w = (to_dev(np.concatenate([w.reshape(-1) for w in inp["conv_w"]])), kappa)
         phi_act = to_dev(np.ascontiguousarray(inp["phi_act"].T))
         b_act = to_dev(inp["b_act"])
         r = len(inp["kappa"])
@@ -501,9 +502,10 @@ def run_secondary(args, local):
 
 
 # ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the current
-# kernels on this workload (profiles/*.txt); None until captured for the
-# kernel version in the tree.
-TRAFFIC = {}
+# kernels, from one --set full capture at T=6144 scaled to T=8192 by the token
+# count (profiles/mhc_pre_tc_T6144_n4_C4096_full.md, mhc_post_...).  Set to
+# None whenever a kernel changes after its capture.
+TRAFFIC = {"mhc_pre": 343.3e6, "mhc_post": 541.4e6}
 
 
 def main(argv=None):
