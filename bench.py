@@ -143,6 +143,12 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def job_throughput(world: int, tokens_per_rank: int, steps: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every rank processes its own tokens_per_rank per step
+    (weak scaling); the time is the maximum over ranks of the timed region."""
+    return world * tokens_per_rank * steps / (ms_max / 1e3)
+
+
 def barrier(world: int, device=None):
     if world > 1:
         import torch.distributed as dist
@@ -285,7 +291,7 @@ def run_ours(args, world, rank, local):
     pre_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
     post_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
     ms_per_step = ms / K
-    value = world * T * K / (ms / 1e3)
+    value = job_throughput(world, T, K, ms)
 
     # the CUDA-core (FMA) projection path on the same inputs, for comparison
     fma_ms = None
@@ -336,7 +342,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize(device)
     barrier(world, device)
     e2e_ms = max_over_ranks(s2.elapsed_time(e2), world, device)
-    e2e_value = world * T * Ke / (e2e_ms / 1e3)
+    e2e_value = job_throughput(world, T, Ke, e2e_ms)
 
     # --- roofline of the dominant kernel
     peak, peak_src = measured_peak()
