@@ -48,6 +48,8 @@ struct RouteArgs {
     void* x_in; float* H_pre; float* score; int32_t* idx; float* w;
 };
 mhc_status launch_route(const RouteArgs& a, cudaStream_t s);
+bool route_tc_supported(const RouteArgs& a);
+mhc_status launch_route_tc(const RouteArgs& a, cudaStream_t s);
 
 struct BwdArgs {
     const void* X; const void* F; const void* phi; mhc_dtype dt; float alpha[3]; const float* b;

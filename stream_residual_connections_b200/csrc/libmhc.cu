@@ -7,5 +7,6 @@
 #include "xhc_conv_gs.cu"
 #include "xhc_update.cu"
 #include "xhc_route.cu"
+#include "xhc_route_tc.cu"
 #include "mhc_bwd.cu"
 #include "mhc_bwd_noalloc.cu"

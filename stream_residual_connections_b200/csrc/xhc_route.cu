@@ -127,6 +127,14 @@ static mhc_status launch_nmax(const RouteArgs& a, cudaStream_t s)
 
 mhc_status launch_route(const RouteArgs& a, cudaStream_t s)
 {
+    // the tensor-core path (xhc_route_tc.cu) where it applies, unless the caller chose the
+    // CUDA-core path with mhc_set_path
+    const bool tc_ok = route_tc_supported(a);
+    if (g_pre_path == MHC_PATH_TENSOR && !tc_ok) {
+        set_error("xhc_route: the tensor-core path needs bf16, N in {4, 8, 12, 16} and C %% 512 == 0");
+        return MHC_ERR_UNSUPPORTED;
+    }
+    if (tc_ok && g_pre_path != MHC_PATH_FMA) return launch_route_tc(a, s);
     if (a.N <= 8) return xroute::launch_nmax<8>(a, s);
     if (a.N <= 16) return xroute::launch_nmax<16>(a, s);
     return xroute::launch_nmax<32>(a, s);

@@ -220,9 +220,62 @@ def test_route_ties_go_to_the_lower_index():
     np.testing.assert_allclose(w.cpu().numpy()[:, m:], 0.5)
 
 
+@pytest.fixture
+def route_path():
+    yield
+    M.mhc_set_path(M.MHC_PATH_AUTO)
+
+
+@pytest.mark.parametrize("T,N,k,m,C", [(100, 16, 4, 2, 512), (33, 8, 4, 2, 1024), (65, 12, 5, 1, 512),
+                                       (7, 4, 2, 0, 512), (300, 16, 8, 3, 2048), (40, 16, 2, 2, 512),
+                                       (31, 8, 8, 2, 512), (1, 16, 4, 2, 1536)])
+def test_route_tensor_core_path_matches_oracle(T, N, k, m, C, route_path):
+    """TMA + tcgen05 route (groups of 4 streams, 32-token tiles): N = 4, 8, 12, 16;
+    ragged last tile; m = 0; k = m (no routed pick); k = N (every stream active)."""
+    M.mhc_set_path(M.MHC_PATH_TENSOR)
+    inp = gapped(synth.xhc_inputs(T, N=N, k=k, m=m, C=C, seed=750 + T + N + C))
+    _route_check(inp)
+
+
+def test_route_tensor_and_cuda_core_paths_agree(route_path):
+    inp = gapped(synth.xhc_inputs(200, N=16, k=4, m=2, C=1024, seed=77))
+    Xd, phiT, b = dev(inp["X"]), dev(np.ascontiguousarray(inp["phi_read"].T)), torch.from_numpy(inp["b_read"]).cuda()
+    outs = {}
+    for path in (M.MHC_PATH_FMA, M.MHC_PATH_TENSOR):
+        M.mhc_set_path(path)
+        outs[path] = [host(t) for t in M.xhc_route(Xd, phiT, inp["alpha_read"], b, inp["k"], inp["m"], inp["eps"])]
+    a, t = outs[M.MHC_PATH_FMA], outs[M.MHC_PATH_TENSOR]
+    np.testing.assert_array_equal(a[3], t[3])                # idx
+    for j, name in ((1, "H_pre"), (2, "score"), (4, "w")):
+        assert np.abs(a[j] - t[j]).max() <= 2e-6, name
+
+
+def test_route_tensor_core_ties_go_to_the_lower_index(route_path):
+    M.mhc_set_path(M.MHC_PATH_TENSOR)
+    T, N, k, m, C = 40, 16, 5, 2, 512
+    inp = synth.xhc_inputs(T, N=N, k=k, m=m, C=C, seed=19)
+    b = inp["b_read"].copy()
+    b[N:] = 0.0                                          # every routed score sigma(0)
+    _, _, sc, idx, w = M.xhc_route(dev(inp["X"]), dev(np.ascontiguousarray(inp["phi_read"].T)),
+                                   [0.0, 0.0], torch.from_numpy(b).cuda(), k, m)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(idx.cpu().numpy(), np.tile(np.arange(k, dtype=np.int32), (T, 1)))
+    np.testing.assert_allclose(w.cpu().numpy()[:, m:], 0.5)
+
+
+def test_route_tensor_core_path_rejects_unsupported_calls(route_path):
+    M.mhc_set_path(M.MHC_PATH_TENSOR)
+    inp = synth.xhc_inputs(8, N=6, k=3, m=1, C=512, seed=20)       # N not a multiple of 4
+    with pytest.raises(M.MhcError) as e:
+        M.xhc_route(dev(inp["X"]), dev(np.ascontiguousarray(inp["phi_read"].T)), inp["alpha_read"],
+                    torch.from_numpy(inp["b_read"]).cuda(), inp["k"], inp["m"])
+    assert e.value.status == M.MHC_ERR_UNSUPPORTED
+
+
 def test_route_xhc_workload_sampled():
-    """T=8192, N=16, k=4, m=2, C=2048: all tokens routed on the GPU, 64 sampled tokens
-    compared (score gaps > 1e-4 after redrawing)."""
+    """T=8192, N=16, k=4, m=2, C=2048 (the tensor-core path, as the benchmark runs it):
+    all tokens routed on the GPU, 64 sampled tokens compared (score gaps > 1e-4 after
+    redrawing)."""
     inp, _ = xhc_full()
     rng = np.random.default_rng(3)
     toks = np.unique(np.concatenate([[0, 8191], rng.choice(8192, 62, replace=False)]))
