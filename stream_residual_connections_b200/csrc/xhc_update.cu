@@ -11,7 +11,10 @@
 // One block of 256 threads per tile of 16 tokens.  Phase 1 projects the
 // gathered rows on CUDA cores: K = kC is walked in chunks of 64 staged in
 // shared memory (the X_act chunk of all 16 tokens and the phi_act^T chunk,
-// double buffered), 16 threads per token each owning up to 4 logits.
+// double buffered; the next chunk's loads are in flight in registers while
+// the current one is multiplied), 16 threads per token each owning up to 4
+// logits; phi_act^T is stored as float4 per (k quad, logit), so the 16 threads
+// of a token read consecutive 16-byte words.
 // Phase 2: per-token coefficients (one thread per token).  Phase 3: the mix,
 // reading X_act again (the block read it moments ago, so from L2) and V,
 // writing the k updated rows in place.
@@ -63,7 +66,7 @@ update_kernel(TX* X, const float* __restrict__ V, const int32_t* __restrict__ id
     constexpr int PPT = (PA + TPT - 1) / TPT;     // logits per thread
     static_assert(PPT <= 4, "at most 64 logits");
     __shared__ __align__(16) float xs[2][TT][KCH];
-    __shared__ __align__(16) float ps[2][PA][KCH];
+    __shared__ __align__(16) float4 ps[2][KCH / 4][PA];   // phi_act^T chunk, (k quad, logit): conflict-free
     __shared__ float ssq[TT];
     __shared__ float logit[TT][PA];
     __shared__ float hres[TT][K][K];
@@ -94,36 +97,60 @@ update_kernel(TX* X, const float* __restrict__ V, const int32_t* __restrict__ id
 #pragma unroll
     for (int q = 0; q < PPT; ++q) acc[q] = 0.0f;
     float ss = 0.0f;
-    auto stage = [&](int ch, int buf) {
+    // chunk staging through registers: the loads of chunk ch+1 are in flight while
+    // chunk ch is multiplied out of shared memory
+    constexpr int XV = TT * (KCH / 8), PV = PA * (KCH / 8);       // 8-element vectors per chunk
+    constexpr int XPT = (XV + THREADS - 1) / THREADS, PPV = (PV + THREADS - 1) / THREADS;
+    float xr8[XPT][8], pr8[PPV][8];
+    auto fetch = [&](int ch) {
         const int64_t k0 = int64_t(ch) * KCH;
-        // X_act chunk: TT tokens x KCH (8-element vectors; a chunk never straddles
-        // two slots because C % KCH == 0)
-        for (int e = tid; e < TT * (KCH / 8); e += THREADS) {
-            const int tt = e / (KCH / 8), v = e % (KCH / 8);
-            const int64_t k = k0 + v * 8;
-            const int l = int(k / C), c = int(k - int64_t(l) * C);
-            float f[8];
-            if (sok[tt]) load8<TX>(X + ((t0 + tt) * N + sidx[tt][l]) * int64_t(C) + c, f);
-            else {
 #pragma unroll
-                for (int q = 0; q < 8; ++q) f[q] = 0.0f;
+        for (int u = 0; u < XPT; ++u) {
+            const int e = tid + u * THREADS;
+            if (e < XV) {
+                // X_act chunk: TT tokens x KCH (a chunk never straddles two slots: C % KCH == 0)
+                const int tt = e / (KCH / 8), v = e % (KCH / 8);
+                const int64_t k = k0 + v * 8;
+                const int l = int(k / C), c = int(k - int64_t(l) * C);
+                if (sok[tt]) load8<TX>(X + ((t0 + tt) * N + sidx[tt][l]) * int64_t(C) + c, xr8[u]);
+                else {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) xr8[u][q] = 0.0f;
+                }
             }
-#pragma unroll
-            for (int q = 0; q < 8; ++q) xs[buf][tt][v * 8 + q] = f[q];
         }
-        for (int e = tid; e < PA * (KCH / 8); e += THREADS) {
-            const int p = e / (KCH / 8), v = e % (KCH / 8);
-            float f[8];
-            load8<TX>(phiT + int64_t(p) * KT + k0 + v * 8, f);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) ps[buf][p][v * 8 + q] = f[q];
+        for (int u = 0; u < PPV; ++u) {
+            const int e = tid + u * THREADS;
+            if (e < PV) load8<TX>(phiT + int64_t(e / (KCH / 8)) * KT + k0 + (e % (KCH / 8)) * 8, pr8[u]);
         }
     };
-    stage(0, 0);
+    auto put = [&](int buf) {
+#pragma unroll
+        for (int u = 0; u < XPT; ++u) {
+            const int e = tid + u * THREADS;
+            if (e < XV) {
+                const int tt = e / (KCH / 8), v = e % (KCH / 8);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) xs[buf][tt][v * 8 + q] = xr8[u][q];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < PPV; ++u) {
+            const int e = tid + u * THREADS;
+            if (e < PV) {
+                const int p = e / (KCH / 8), v = e % (KCH / 8);
+                ps[buf][2 * v][p] = make_float4(pr8[u][0], pr8[u][1], pr8[u][2], pr8[u][3]);
+                ps[buf][2 * v + 1][p] = make_float4(pr8[u][4], pr8[u][5], pr8[u][6], pr8[u][7]);
+            }
+        }
+    };
+    fetch(0);
+    put(0);
     __syncthreads();
     for (int ch = 0; ch < nchunks; ++ch) {
         const int buf = ch & 1;
-        if (ch + 1 < nchunks) stage(ch + 1, buf ^ 1);
+        if (ch + 1 < nchunks) fetch(ch + 1);
         const float* xr = xs[buf][my_t];
 #pragma unroll 4
         for (int kk = 0; kk < KCH; kk += 4) {
@@ -136,7 +163,7 @@ update_kernel(TX* X, const float* __restrict__ V, const int32_t* __restrict__ id
             for (int q = 0; q < PPT; ++q) {
                 const int p = sub + q * TPT;
                 if (p < PA) {
-                    const float4 p4 = *reinterpret_cast<const float4*>(&ps[buf][p][kk]);
+                    const float4 p4 = ps[buf][kk / 4][p];
                     acc[q] = fmaf(x4.x, p4.x, acc[q]);
                     acc[q] = fmaf(x4.y, p4.y, acc[q]);
                     acc[q] = fmaf(x4.z, p4.z, acc[q]);
@@ -144,6 +171,7 @@ update_kernel(TX* X, const float* __restrict__ V, const int32_t* __restrict__ id
                 }
             }
         }
+        if (ch + 1 < nchunks) put(buf ^ 1);
         __syncthreads();
     }
 #pragma unroll
