@@ -56,7 +56,9 @@ struct BwdArgs {
     const void* dXn; const void* dxin; int64_t T; int n; int C; int t_iters; float eps;
     void* dX; void* dF; float* dphi; float* dalpha; float* db;
     float* records; float* u_scratch; float* r_scratch;   // carved from the caller's workspace
+    float* dphi_part;                                     // [segments][P][nC] when segments > 1
 };
+int backward_b3_segments(int64_t T);
 size_t backward_record_stride(int n);            // floats per token record (0: unsupported n)
 mhc_status launch_backward(const BwdArgs& a, cudaStream_t s);
 

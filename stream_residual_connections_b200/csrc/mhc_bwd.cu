@@ -18,10 +18,13 @@
 //   B1  one block per token: the P dot products, dF, and the per-token
 //       coefficient gradients (Sinkhorn forward trace kept in shared memory,
 //       then walked backwards) -> workspace
-//   B2  dX over 16-token x 64-channel tiles (all streams), phi^T chunk in
-//       shared memory
-//   B3  dphi^T[p][k] = sum_t dd[t][p] x[t][k] over 64-column slabs of all
-//       tokens (deterministic order), and db / dalpha by per-output tree sums
+//   B2  dX over 64-token x 64-channel tiles (all streams), phi^T chunk in
+//       shared memory (read once per 64 tokens)
+//   B3  dphi^T[p][k] = sum_t dd[t][p] x[t][k]: blocks of 64 columns x one of S
+//       token segments (S = ceil(T / 512), at most 16), 64-token chunks staged
+//       through registers; with S > 1 the per-segment sums go to the workspace
+//       and B3R adds them in segment order (deterministic); db / dalpha by
+//       per-output tree sums
 #include "common.cuh"
 #include "internal.h"
 
@@ -248,7 +251,7 @@ b1_kernel(const TX* __restrict__ X, const TX* __restrict__ F, const TX* __restri
 }
 
 // ---------------------------------------------------------------- B2
-constexpr int B2_T = 16, B2_C = 64;
+constexpr int B2_T = 64, B2_C = 64, B2_SUB = 16;   // tokens per block; per pass of the 128 threads
 
 template <int N, typename TX>
 __global__ void __launch_bounds__(128)
@@ -282,9 +285,10 @@ b2_kernel(const TX* __restrict__ X, const TX* __restrict__ dXn, const TX* __rest
         shp[tt][q] = (t0 + tt < T) ? ws[(t0 + tt) * L::STRIDE + L::HPRE + q] : 0.0f;
     }
     __syncthreads();
-    const int tt = tid / (B2_C / 8), v = tid % (B2_C / 8);
+    const int v = tid % (B2_C / 8);
+    for (int tt = tid / (B2_C / 8); tt < B2_T; tt += B2_SUB) {
     const int64_t t = t0 + tt;
-    if (t >= T) return;
+    if (t >= T) break;
     const int c = c0 + v * 8;
     float g[N][8], x[N][8], gi[8];
 #pragma unroll
@@ -312,38 +316,78 @@ b2_kernel(const TX* __restrict__ X, const TX* __restrict__ dXn, const TX* __rest
         }
         store8<TX>(dX + (t * N + j) * C + c, o);
     }
+    }
 }
 
 // ---------------------------------------------------------------- B3
-constexpr int B3_K = 64, B3_T = 64;
+constexpr int B3_K = 64, B3_T = 64, B3_SEG_MIN = 512, B3_MAX_SEGS = 16;
 
+// token segments of B3 for T tokens (the workspace holds S - 1 extra dphi copies
+// when S > 1; see mhc_backward_workspace_bytes)
+inline int b3_segments(int64_t T)
+{
+    const int64_t s = (T + B3_SEG_MIN - 1) / B3_SEG_MIN;
+    return int(s < 1 ? 1 : (s > B3_MAX_SEGS ? B3_MAX_SEGS : s));
+}
+
+// block (k slab, segment): out[p][k0 + kk] = sum over the segment's tokens of
+// dd[t][p] * x[t][k0 + kk]; out is dphi^T (one segment) or the segment's slice
+// of the partial sums
 template <int N, typename TX>
 __global__ void __launch_bounds__(256)
-b3_kernel(const TX* __restrict__ X, const float* __restrict__ ws, int64_t T, int C, float* __restrict__ dphiT)
+b3_kernel(const TX* __restrict__ X, const float* __restrict__ ws, int64_t T, int C, int64_t seg_len,
+          float* __restrict__ out)
 {
     using L = WS<N>;
     constexpr int P = L::P;
     constexpr int PG = 256 / B3_K;                 // p groups
     constexpr int PPT = (P + PG - 1) / PG;         // p per thread
+    constexpr int XV = B3_T * (B3_K / 8);          // 8-element X vectors per chunk (2 per thread)
+    constexpr int DV = B3_T * P;                   // dd values per chunk
+    constexpr int DPT = (DV + 255) / 256;
     __shared__ __align__(16) float sx[B3_T][B3_K];
     __shared__ float sdd[B3_T][P];
     const int64_t K = int64_t(N) * C;
     const int64_t k0 = int64_t(blockIdx.x) * B3_K;
+    const int64_t ta = int64_t(blockIdx.y) * seg_len;
+    const int64_t tb = ta + seg_len < T ? ta + seg_len : T;
     const int tid = threadIdx.x, kk = tid % B3_K, pg = tid / B3_K;
     float acc[PPT];
 #pragma unroll
     for (int q = 0; q < PPT; ++q) acc[q] = 0.0f;
-    for (int64_t t0 = 0; t0 < T; t0 += B3_T) {
-        __syncthreads();
-        for (int e = tid; e < B3_T * B3_K; e += 256) {
-            const int tt = e / B3_K, c = e % B3_K;
-            sx[tt][c] = (t0 + tt < T && k0 + c < K) ? to_f32(X[(t0 + tt) * K + k0 + c]) : 0.0f;
+    float xr[XV / 256][8], dr[DPT];
+    auto fetch = [&](int64_t t0) {
+#pragma unroll
+        for (int u = 0; u < XV / 256; ++u) {
+            const int e = tid + u * 256, tt = e / (B3_K / 8), vv = e % (B3_K / 8);
+            if (t0 + tt < tb) load8<TX>(X + (t0 + tt) * K + k0 + vv * 8, xr[u]);
+            else {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) xr[u][q] = 0.0f;
+            }
         }
-        for (int e = tid; e < B3_T * P; e += 256) {
-            const int tt = e / P, p = e % P;
-            sdd[tt][p] = (t0 + tt < T) ? ws[(t0 + tt) * L::STRIDE + L::DD + p] : 0.0f;
+#pragma unroll
+        for (int u = 0; u < DPT; ++u) {
+            const int e = tid + u * 256, tt = e / P, p = e % P;
+            dr[u] = (e < DV && t0 + tt < tb) ? ws[(t0 + tt) * L::STRIDE + L::DD + p] : 0.0f;
+        }
+    };
+    if (ta < tb) fetch(ta);
+    for (int64_t t0 = ta; t0 < tb; t0 += B3_T) {
+        __syncthreads();                           // the previous chunk is consumed
+#pragma unroll
+        for (int u = 0; u < XV / 256; ++u) {
+            const int e = tid + u * 256, tt = e / (B3_K / 8), vv = e % (B3_K / 8);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) sx[tt][vv * 8 + q] = xr[u][q];
+        }
+#pragma unroll
+        for (int u = 0; u < DPT; ++u) {
+            const int e = tid + u * 256;
+            if (e < DV) sdd[e / P][e % P] = dr[u];
         }
         __syncthreads();
+        if (t0 + B3_T < tb) fetch(t0 + B3_T);     // next chunk in flight during the products
 #pragma unroll 4
         for (int tt = 0; tt < B3_T; ++tt) {
             const float xv = sx[tt][kk];
@@ -354,13 +398,23 @@ b3_kernel(const TX* __restrict__ X, const float* __restrict__ ws, int64_t T, int
             }
         }
     }
-    if (k0 + kk < K) {
+    float* o = out + int64_t(blockIdx.y) * P * K;
 #pragma unroll
-        for (int q = 0; q < PPT; ++q) {
-            const int p = pg + q * PG;
-            if (p < P) dphiT[int64_t(p) * K + k0 + kk] = acc[q];
-        }
+    for (int q = 0; q < PPT; ++q) {
+        const int p = pg + q * PG;
+        if (p < P) o[int64_t(p) * K + k0 + kk] = acc[q];
     }
+}
+
+// dphi^T[i] = sum_s part[s][i] in segment order
+__global__ void __launch_bounds__(256)
+b3r_kernel(const float* __restrict__ part, int segs, int64_t count, float* __restrict__ dphiT)
+{
+    const int64_t i = int64_t(blockIdx.x) * 256 + threadIdx.x;
+    if (i >= count) return;
+    float s = 0.0f;
+    for (int q = 0; q < segs; ++q) s += part[int64_t(q) * count + i];
+    dphiT[i] = s;
 }
 
 // one block per output: db[p] = sum_t dz[t][p]; dalpha[s] = sum_t da[t][s]
@@ -414,15 +468,25 @@ static mhc_status run(const BwdArgs& a, cudaStream_t s)
     st = launch_status("mhc_backward B2 kernel");
     if (st != MHC_OK) return st;
     const int64_t K = int64_t(N) * a.C;
-    b3_kernel<N, TX><<<dim3(unsigned((K + B3_K - 1) / B3_K)), 256, 0, s>>>(
-        static_cast<const TX*>(a.X), ws, a.T, a.C, a.dphi);
+    const int segs = b3_segments(a.T);
+    const int64_t seg_len = ((a.T + segs - 1) / segs + B3_T - 1) / B3_T * B3_T;
+    b3_kernel<N, TX><<<dim3(unsigned(K / B3_K), unsigned(segs)), 256, 0, s>>>(
+        static_cast<const TX*>(a.X), ws, a.T, a.C, seg_len, segs > 1 ? a.dphi_part : a.dphi);
     st = launch_status("mhc_backward B3 kernel");
     if (st != MHC_OK) return st;
+    if (segs > 1) {
+        const int64_t count = int64_t(P) * K;
+        b3r_kernel<<<dim3(unsigned((count + 255) / 256)), 256, 0, s>>>(a.dphi_part, segs, count, a.dphi);
+        st = launch_status("mhc_backward B3 reduction kernel");
+        if (st != MHC_OK) return st;
+    }
     bsum_kernel<N><<<dim3(unsigned(P + 3)), 256, 0, s>>>(ws, a.T, a.db, a.dalpha);
     return launch_status("mhc_backward reduction kernel");
 }
 
 }  // namespace bwd
+
+int backward_b3_segments(int64_t T) { return bwd::b3_segments(T); }
 
 size_t backward_record_stride(int n)
 {
