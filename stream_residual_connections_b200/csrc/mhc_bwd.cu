@@ -300,19 +300,32 @@ b2_kernel(const TX* __restrict__ X, const TX* __restrict__ dXn, const TX* __rest
     const float* hres = sco[tt];              // [N][N]
     const float cr = sco[tt][N * N];
     const float* hpre = shp[tt];
+    float dd[P];                              // this token's dd in registers
+#pragma unroll
+    for (int p = 0; p < P; ++p) dd[p] = sdd[tt][p];
 #pragma unroll
     for (int j = 0; j < N; ++j) {
         const float hpj = hpre[j];
+        // (phi dd)_j for the thread's 8 channels: two 16-byte phi reads per logit
+        float pr[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pr[e] = 0.0f;
+#pragma unroll
+        for (int p = 0; p < P; ++p) {
+            const float4 lo = *reinterpret_cast<const float4*>(&sphi[p][j][v * 8]);
+            const float4 hi = *reinterpret_cast<const float4*>(&sphi[p][j][v * 8 + 4]);
+            pr[0] = fmaf(lo.x, dd[p], pr[0]); pr[1] = fmaf(lo.y, dd[p], pr[1]);
+            pr[2] = fmaf(lo.z, dd[p], pr[2]); pr[3] = fmaf(lo.w, dd[p], pr[3]);
+            pr[4] = fmaf(hi.x, dd[p], pr[4]); pr[5] = fmaf(hi.y, dd[p], pr[5]);
+            pr[6] = fmaf(hi.z, dd[p], pr[6]); pr[7] = fmaf(hi.w, dd[p], pr[7]);
+        }
         float o[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             float s = hpj * gi[e];
 #pragma unroll
             for (int i = 0; i < N; ++i) s = fmaf(hres[i * N + j], g[i][e], s);
-            float pr = 0.0f;
-#pragma unroll
-            for (int p = 0; p < P; ++p) pr = fmaf(sphi[p][j][v * 8 + e], sdd[tt][p], pr);
-            o[e] = s + pr + cr * x[j][e];
+            o[e] = s + pr[e] + cr * x[j][e];
         }
         store8<TX>(dX + (t * N + j) * C + c, o);
     }
