@@ -15,9 +15,10 @@
 // v_j = 0 and contributes nothing afterwards, as in MGS.
 //
 // One block of 256 threads per tile of 8 consecutive tokens; a thread owns
-// 8 channels at a time.  Pass 1 accumulates the Gram partials, the block
-// reduces them, pass 2 recomputes the components (the input rows and weights
-// are L1/L2-resident) and writes V in fp32.
+// 8 channels at a time.  Pass 1 forms the components (each input row loaded
+// once for all convolutions; rows and weights are L1/L2-resident) and
+// accumulates the Gram partials, the block reduces them, pass 2 writes V in
+// fp32 from the components kept in registers (C <= 2048) or recomputed.
 #include "common.cuh"
 #include "internal.h"
 
@@ -47,7 +48,8 @@ struct Params {
     int64_t woff[MAXR];
 };
 
-// a[0..R][8] for token t, channels c..c+7
+// a[0..R][8] for token t, channels c..c+7.  Each of the max kappa input rows
+// out[t-s] is loaded once and feeds every convolution that reaches it.
 template <int R, typename TF>
 __device__ __forceinline__ void components(const TF* __restrict__ F, const float* __restrict__ W,
                                            const Params& prm, int64_t t, int64_t pos, int C, int c,
@@ -55,27 +57,39 @@ __device__ __forceinline__ void components(const TF* __restrict__ F, const float
 {
     load8<TF>(F + t * C + c, a[0]);
 #pragma unroll
-    for (int j = 0; j < R; ++j) {
+    for (int j = 0; j < R; ++j)
 #pragma unroll
         for (int e = 0; e < 8; ++e) a[j + 1][e] = 0.0f;
-        const int kj = prm.kap[j];
-        for (int s = 0; s < kj && s <= pos; ++s) {
-            float f[8], w0[4], w1[4];
-            load8<TF>(F + (t - s) * C + c, f);
-            const float* wp = W + prm.woff[j] + int64_t(s) * C + c;
-            load16<false>(wp, w0);
-            load16<false>(wp + 4, w1);
+    int kmax = 0;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                a[j + 1][e] = fmaf(w0[e], f[e], a[j + 1][e]);
-                a[j + 1][4 + e] = fmaf(w1[e], f[4 + e], a[j + 1][4 + e]);
+    for (int j = 0; j < R; ++j) kmax = prm.kap[j] > kmax ? prm.kap[j] : kmax;
+    for (int s = 0; s < kmax && s <= pos; ++s) {
+        float f[8];
+        if (s == 0) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = a[0][e];
+        } else {
+            load8<TF>(F + (t - s) * C + c, f);
+        }
+#pragma unroll
+        for (int j = 0; j < R; ++j) {
+            if (s < prm.kap[j]) {
+                float w0[4], w1[4];
+                const float* wp = W + prm.woff[j] + int64_t(s) * C + c;
+                load16<false>(wp, w0);
+                load16<false>(wp + 4, w1);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    a[j + 1][e] = fmaf(w0[e], f[e], a[j + 1][e]);
+                    a[j + 1][4 + e] = fmaf(w1[e], f[4 + e], a[j + 1][4 + e]);
+                }
             }
         }
     }
 }
 
 template <int R, typename TF>
-__global__ void __launch_bounds__(THREADS)
+__global__ void __launch_bounds__(THREADS, 2)
 conv_gs_kernel(const TF* __restrict__ F, const float* __restrict__ W, Params prm, int64_t T, int C,
                int64_t seq_len, float* __restrict__ V)
 {
@@ -85,6 +99,10 @@ conv_gs_kernel(const TF* __restrict__ F, const float* __restrict__ W, Params prm
     __shared__ float Gs[NG];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int CV = C / 8;
+    // a thread that owns a single channel vector keeps its components between the
+    // Gram pass and the output pass; otherwise the output pass recomputes them
+    const bool one = CV <= THREADS;
+    float keep[KR][8];
     for (int tt = 0; tt < TILE; ++tt) {
         const int64_t t = int64_t(blockIdx.x) * TILE + tt;
         if (t >= T) break;                       // uniform across the block
@@ -95,6 +113,12 @@ conv_gs_kernel(const TF* __restrict__ F, const float* __restrict__ W, Params prm
         for (int v = threadIdx.x; v < CV; v += THREADS) {
             float a[KR][8];
             components<R, TF>(F, W, prm, t, pos, C, v * 8, a);
+            if (one) {
+#pragma unroll
+                for (int i = 0; i < KR; ++i)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) keep[i][e] = a[i][e];
+            }
             int q = 0;
 #pragma unroll
             for (int i = 0; i < KR; ++i)
@@ -156,7 +180,14 @@ conv_gs_kernel(const TF* __restrict__ F, const float* __restrict__ W, Params prm
         }
         for (int v = threadIdx.x; v < CV; v += THREADS) {
             float a[KR][8];
-            components<R, TF>(F, W, prm, t, pos, C, v * 8, a);
+            if (one) {
+#pragma unroll
+                for (int i = 0; i < KR; ++i)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) a[i][e] = keep[i][e];
+            } else {
+                components<R, TF>(F, W, prm, t, pos, C, v * 8, a);
+            }
 #pragma unroll
             for (int j = 0; j < KR; ++j) {
                 float o[8];
