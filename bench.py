@@ -486,6 +486,33 @@ def run_secondary(args, local):
         for f in launches():
             f()
     torch.cuda.synchronize(device)
+    # the fp64 oracle on a bounded sample of the same workload's tokens (host cores)
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        oracle.lib()
+        if args.workload == "xhc":
+            def oracle_step(S):
+                rt = oracle.xhc_route(inp["X"][:S], inp["phi_read"], inp["alpha_read"], inp["b_read"], k, m,
+                                      inp["eps"])
+                V0 = oracle.xhc_conv_gs(inp["F"][:S], inp["conv_w"], seq_len=T)
+                oracle.xhc_sparse_update(inp["X"][:S], V0, rt["idx"], rt["w"], inp["phi_act"], inp["alpha_act"],
+                                         inp["b_act"], inp["t_iters"], inp["eps"])
+            what = "xhc_route + xhc_conv_gs + xhc_sparse_update"
+        else:
+            def oracle_step(S):
+                oracle.mhc_backward(inp["X"][:S], inp["F"][:S], inp["phi"], inp["alpha"], inp["b"],
+                                    inp["dX_next"][:S], inp["dx_in"][:S], 20, 1e-6)
+            what = "mhc_backward"
+        t_a = time.perf_counter()
+        oracle_step(4)
+        per_tok = (time.perf_counter() - t_a) / 4
+        S = int(max(4, min(T, args.cpu_seconds / max(per_tok, 1e-9))))
+        t_a = time.perf_counter()
+        oracle_step(S)
+        dt = time.perf_counter() - t_a
+        cpu = {"value": S / dt, "unit": "tokens/s", "cores": int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1)),
+               "kind": "oracle", "sample": f"first {S} tokens of the same workload, fp64 oracle ({what})"}
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
@@ -504,7 +531,7 @@ def run_secondary(args, local):
         rows[name] = {"ms": kms, "algorithmic_bytes": nbytes[name], "achieved_gbs": gbs, "frac": gbs / peak}
     print(json.dumps({"workload": args.workload, "config": desc, "steps": K, "warmup": args.warmup,
                       "ms_per_step": ms, "tokens_per_s": T / (ms / 1e3), "kernels": rows, "peak_gbs": peak,
-                      "peak_source": peak_src}), flush=True)
+                      "peak_source": peak_src, "cpu_baseline": cpu}), flush=True)
 
 
 # ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the current
