@@ -268,9 +268,13 @@ b2_kernel(const TX* __restrict__ X, const TX* __restrict__ dXn, const TX* __rest
     const int c0 = blockIdx.y * B2_C;
     const int64_t K = int64_t(N) * C;
     const int tid = threadIdx.x;
+    // channel c of the slice is stored at float4 slot (c / 8) for c % 8 < 4 and at slot
+    // 8 + c / 8 otherwise, so the 8 lanes that read a thread's 8 channels read
+    // 128 contiguous bytes (no bank conflict)
     for (int e = tid; e < P * N * B2_C; e += 128) {
         const int p = e / (N * B2_C), rem = e % (N * B2_C), j = rem / B2_C, c = rem % B2_C;
-        sphi[p][j][c] = to_f32(phiT[int64_t(p) * K + int64_t(j) * C + c0 + c]);
+        const int cs = (c & 4) ? 32 + (c >> 3) * 4 + (c & 3) : (c >> 3) * 4 + (c & 3);
+        sphi[p][j][cs] = to_f32(phiT[int64_t(p) * K + int64_t(j) * C + c0 + c]);
     }
     for (int e = tid; e < B2_T * P; e += 128) {
         const int tt = e / P, p = e % P;
@@ -312,8 +316,8 @@ b2_kernel(const TX* __restrict__ X, const TX* __restrict__ dXn, const TX* __rest
         for (int e = 0; e < 8; ++e) pr[e] = 0.0f;
 #pragma unroll
         for (int p = 0; p < P; ++p) {
-            const float4 lo = *reinterpret_cast<const float4*>(&sphi[p][j][v * 8]);
-            const float4 hi = *reinterpret_cast<const float4*>(&sphi[p][j][v * 8 + 4]);
+            const float4 lo = *reinterpret_cast<const float4*>(&sphi[p][j][v * 4]);
+            const float4 hi = *reinterpret_cast<const float4*>(&sphi[p][j][32 + v * 4]);
             pr[0] = fmaf(lo.x, dd[p], pr[0]); pr[1] = fmaf(lo.y, dd[p], pr[1]);
             pr[2] = fmaf(lo.z, dd[p], pr[2]); pr[3] = fmaf(lo.w, dd[p], pr[3]);
             pr[4] = fmaf(hi.x, dd[p], pr[4]); pr[5] = fmaf(hi.y, dd[p], pr[5]);
@@ -353,21 +357,27 @@ b3_kernel(const TX* __restrict__ X, const float* __restrict__ ws, int64_t T, int
 {
     using L = WS<N>;
     constexpr int P = L::P;
-    constexpr int PG = 256 / B3_K;                 // p groups
-    constexpr int PPT = (P + PG - 1) / PG;         // p per thread
+    constexpr int PP = (P + 15) / 16 * 16;         // logits padded to 16 per row of sdd
+    constexpr int PB = PP / 8;                     // logits per thread (8 logit blocks): even, so
+    static_assert(PB % 2 == 0, "float2 reads of sdd stay 8-byte aligned");
     constexpr int XV = B3_T * (B3_K / 8);          // 8-element X vectors per chunk (2 per thread)
     constexpr int DV = B3_T * P;                   // dd values per chunk
     constexpr int DPT = (DV + 255) / 256;
+    static_assert(256 == 32 * 8, "32 column pairs x 8 logit blocks");
     __shared__ __align__(16) float sx[B3_T][B3_K];
-    __shared__ float sdd[B3_T][P];
+    __shared__ __align__(16) float sdd[B3_T][PP];
     const int64_t K = int64_t(N) * C;
     const int64_t k0 = int64_t(blockIdx.x) * B3_K;
     const int64_t ta = int64_t(blockIdx.y) * seg_len;
     const int64_t tb = ta + seg_len < T ? ta + seg_len : T;
-    const int tid = threadIdx.x, kk = tid % B3_K, pg = tid / B3_K;
-    float acc[PPT];
+    const int tid = threadIdx.x;
+    const int kk = tid & 31;                       // columns kk and kk + 32 of the slab
+    const int pb = tid >> 5;                       // logits [pb * PB, pb * PB + PB)
+    float acc[2][PB];
 #pragma unroll
-    for (int q = 0; q < PPT; ++q) acc[q] = 0.0f;
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < PB; ++q) acc[h][q] = 0.0f;
     float xr[XV / 256][8], dr[DPT];
     auto fetch = [&](int64_t t0) {
 #pragma unroll
@@ -399,23 +409,35 @@ b3_kernel(const TX* __restrict__ X, const float* __restrict__ ws, int64_t T, int
             const int e = tid + u * 256;
             if (e < DV) sdd[e / P][e % P] = dr[u];
         }
+        if (PP > P)
+            for (int e = tid; e < B3_T * (PP - P); e += 256) sdd[e / (PP - P)][P + e % (PP - P)] = 0.0f;
         __syncthreads();
         if (t0 + B3_T < tb) fetch(t0 + B3_T);     // next chunk in flight during the products
 #pragma unroll 4
         for (int tt = 0; tt < B3_T; ++tt) {
-            const float xv = sx[tt][kk];
+            const float x0 = sx[tt][kk], x1 = sx[tt][kk + 32];
+            float dd[PB];
 #pragma unroll
-            for (int q = 0; q < PPT; ++q) {
-                const int p = pg + q * PG;
-                if (p < P) acc[q] = fmaf(sdd[tt][p], xv, acc[q]);
+            for (int q = 0; q < PB; q += 2) {
+                const float2 d2 = *reinterpret_cast<const float2*>(&sdd[tt][pb * PB + q]);
+                dd[q] = d2.x;
+                dd[q + 1] = d2.y;
+            }
+#pragma unroll
+            for (int q = 0; q < PB; ++q) {
+                acc[0][q] = fmaf(dd[q], x0, acc[0][q]);
+                acc[1][q] = fmaf(dd[q], x1, acc[1][q]);
             }
         }
     }
     float* o = out + int64_t(blockIdx.y) * P * K;
 #pragma unroll
-    for (int q = 0; q < PPT; ++q) {
-        const int p = pg + q * PG;
-        if (p < P) o[int64_t(p) * K + k0 + kk] = acc[q];
+    for (int q = 0; q < PB; ++q) {
+        const int p = pb * PB + q;
+        if (p < P) {
+            o[int64_t(p) * K + k0 + kk] = acc[0][q];
+            o[int64_t(p) * K + k0 + kk + 32] = acc[1][q];
+        }
     }
 }
 
