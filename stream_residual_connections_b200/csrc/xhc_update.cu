@@ -66,7 +66,12 @@ update_kernel(TX* X, const float* __restrict__ V, const int32_t* __restrict__ id
     constexpr int PPT = (PA + TPT - 1) / TPT;     // logits per thread
     static_assert(PPT <= 4, "at most 64 logits");
     __shared__ __align__(16) float xs[2][TT][KCH];
-    __shared__ __align__(16) float4 ps[2][KCH / 4][PA];   // phi_act^T chunk, (k quad, logit): conflict-free
+    // phi_act^T chunk as float4 per (k quad, logit); logit p of k quad kq sits at
+    // p ^ ((kq / 2) % 8) of a row padded to a multiple of 8, so that both the
+    // stores (8 lanes: one logit, 8 k quads) and the reads (one k quad, 16
+    // logits) touch distinct banks
+    constexpr int PAP = (PA + 7) / 8 * 8;
+    __shared__ __align__(16) float4 ps[2][KCH / 4][PAP];
     __shared__ float ssq[TT];
     __shared__ float logit[TT][PA];
     __shared__ float hres[TT][K][K];
@@ -140,8 +145,8 @@ update_kernel(TX* X, const float* __restrict__ V, const int32_t* __restrict__ id
             const int e = tid + u * THREADS;
             if (e < PV) {
                 const int p = e / (KCH / 8), v = e % (KCH / 8);
-                ps[buf][2 * v][p] = make_float4(pr8[u][0], pr8[u][1], pr8[u][2], pr8[u][3]);
-                ps[buf][2 * v + 1][p] = make_float4(pr8[u][4], pr8[u][5], pr8[u][6], pr8[u][7]);
+                ps[buf][2 * v][p ^ (v & 7)] = make_float4(pr8[u][0], pr8[u][1], pr8[u][2], pr8[u][3]);
+                ps[buf][2 * v + 1][p ^ (v & 7)] = make_float4(pr8[u][4], pr8[u][5], pr8[u][6], pr8[u][7]);
             }
         }
     };
@@ -163,7 +168,7 @@ update_kernel(TX* X, const float* __restrict__ V, const int32_t* __restrict__ id
             for (int q = 0; q < PPT; ++q) {
                 const int p = sub + q * TPT;
                 if (p < PA) {
-                    const float4 p4 = ps[buf][kk / 4][p];
+                    const float4 p4 = ps[buf][kk / 4][p ^ ((kk / 8) & 7)];
                     acc[q] = fmaf(x4.x, p4.x, acc[q]);
                     acc[q] = fmaf(x4.y, p4.y, acc[q]);
                     acc[q] = fmaf(x4.z, p4.z, acc[q]);
