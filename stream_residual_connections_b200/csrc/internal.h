@@ -41,6 +41,8 @@ struct UpdateArgs {
     float* H_res; float* H_post;
 };
 mhc_status launch_sparse_update(const UpdateArgs& a, cudaStream_t s);
+bool update_tc_supported(const UpdateArgs& a);
+mhc_status launch_update_tc(const UpdateArgs& a, cudaStream_t s);
 
 struct RouteArgs {
     const void* X; mhc_dtype dt; const void* phi; float alpha[2]; const float* b;

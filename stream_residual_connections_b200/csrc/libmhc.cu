@@ -6,6 +6,7 @@
 #include "mhc_pre_tc.cu"
 #include "xhc_conv_gs.cu"
 #include "xhc_update.cu"
+#include "xhc_update_tc.cu"
 #include "xhc_route.cu"
 #include "xhc_route_tc.cu"
 #include "mhc_bwd.cu"

@@ -130,6 +130,17 @@ __device__ __forceinline__ bool warp_wait_sleep(uint64_t* bar, uint32_t parity) 
     return __all_sync(0xffffffffu, mbar_wait_sleep(bar, parity));
 }
 
+// ---------------------------------------------------------------- cp.async
+// 16-byte global -> shared copy; src_bytes < 16 zero-fills the rest (0: all zeros,
+// nothing read), with an L2 cache policy.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes, uint64_t policy) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;"
+                 :: "r"(smem_u32(dst)), "l"(src), "r"(src_bytes), "l"(policy) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");

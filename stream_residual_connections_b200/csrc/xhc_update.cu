@@ -286,6 +286,14 @@ static mhc_status launch_k(const UpdateArgs& a, cudaStream_t s)
 
 mhc_status launch_sparse_update(const UpdateArgs& a, cudaStream_t s)
 {
+    // the tensor-core path (xhc_update_tc.cu) where it applies, unless the caller chose
+    // the CUDA-core path with mhc_set_path
+    const bool tc_ok = update_tc_supported(a);
+    if (g_pre_path == MHC_PATH_TENSOR && !tc_ok) {
+        set_error("xhc_sparse_update: the tensor-core path needs bf16, k = 4, Kr <= 4 and C %% 512 == 0");
+        return MHC_ERR_UNSUPPORTED;
+    }
+    if (tc_ok && g_pre_path != MHC_PATH_FMA) return launch_update_tc(a, s);
     switch (a.k) {
         case 1: return xupd::launch_k<1>(a, s);
         case 2: return xupd::launch_k<2>(a, s);

@@ -135,8 +135,68 @@ def test_sparse_update_out_of_range_index_is_reported_and_token_untouched():
     M.mhc_sync_status()
 
 
+@pytest.mark.parametrize("T,N,m,C,kappa", [(100, 16, 2, 512, (4, 8, 12)), (33, 8, 1, 1024, (4,)),
+                                           (65, 6, 2, 512, (3, 5)), (1, 4, 0, 1536, (4, 8, 12)),
+                                           (300, 16, 3, 2048, (2, 4, 6))])
+def test_sparse_update_tensor_core_path_matches_oracle(T, N, m, C, kappa, update_path):
+    """cp.async gather + TMA + tcgen05 projection for k = 4 active streams; Kr = 2, 3, 4;
+    ragged last tile."""
+    M.mhc_set_path(M.MHC_PATH_TENSOR)
+    inp = synth.xhc_inputs(T, N=N, k=4, m=m, C=C, kappa=kappa, seed=800 + T + N + C)
+    _update_case(inp)
+
+
+def test_sparse_update_tensor_and_cuda_core_paths_agree(update_path):
+    inp = synth.xhc_inputs(96, N=16, k=4, m=2, C=1024, seed=81)
+    rt = _route_ref(inp)
+    V = torch.from_numpy(oracle.xhc_conv_gs(inp["F"], inp["conv_w"]).astype(np.float32)).cuda()
+    args = (V, torch.from_numpy(rt["idx"]).cuda(), torch.from_numpy(rt["w"].astype(np.float32)).cuda(),
+            dev(np.ascontiguousarray(inp["phi_act"].T)), inp["alpha_act"], torch.from_numpy(inp["b_act"]).cuda(),
+            inp["t_iters"], inp["eps"])
+    outs = {}
+    for path in (M.MHC_PATH_FMA, M.MHC_PATH_TENSOR):
+        M.mhc_set_path(path)
+        Xd = dev(inp["X"])
+        _, Hr, Hp = M.xhc_sparse_update(Xd, *args)
+        outs[path] = (host(Xd), host(Hr), host(Hp))
+    a, t = outs[M.MHC_PATH_FMA], outs[M.MHC_PATH_TENSOR]
+    assert np.abs(a[1] - t[1]).max() <= 2e-6 and np.abs(a[2] - t[2]).max() <= 2e-6
+    # bf16 rows: equal up to a rounding flip where the fp32 sums differ in the last bits
+    assert np.abs(a[0] - t[0]).max() <= 2 ** -6 * np.abs(a[0]).max()
+
+
+def test_sparse_update_tensor_core_out_of_range_index_is_reported(update_path):
+    M.mhc_set_path(M.MHC_PATH_TENSOR)
+    T, N, k, C = 40, 8, 4, 512
+    inp = synth.xhc_inputs(T, N=N, k=k, m=2, C=C, seed=17)
+    idx = np.tile(np.array([0, 1, 2, 3], dtype=np.int32), (T, 1))
+    idx[3, 2] = N + 5
+    idx[35, 0] = -1
+    Xd = dev(inp["X"])
+    X0 = host(Xd)
+    V = torch.zeros((T, 4, C), device="cuda")
+    M.xhc_sparse_update(Xd, V, torch.from_numpy(idx).cuda(), torch.ones((T, k), device="cuda"),
+                        dev(np.ascontiguousarray(inp["phi_act"].T)), inp["alpha_act"],
+                        torch.from_numpy(inp["b_act"]).cuda())
+    with pytest.raises(M.MhcError) as e:
+        M.mhc_sync_status()
+    assert e.value.status == M.MHC_ERR_INVALID_ARG
+    got = host(Xd)
+    np.testing.assert_array_equal(got[3], X0[3])
+    np.testing.assert_array_equal(got[35], X0[35])
+    assert not np.array_equal(got[2], X0[2])
+    M.mhc_sync_status()
+
+
+@pytest.fixture
+def update_path():
+    yield
+    M.mhc_set_path(M.MHC_PATH_AUTO)
+
+
 def test_sparse_update_xhc_workload_sampled():
-    """T=8192, N=16, k=4 (m=2), C=2048: the update runs on all tokens; 48 are compared."""
+    """T=8192, N=16, k=4 (m=2), C=2048 (the tensor-core path, as the benchmark runs
+    it): the update runs on all tokens; 48 are compared."""
     inp, rt = xhc_full()
     rng = np.random.default_rng(2)
     toks = np.unique(np.concatenate([[0, 8191], rng.choice(8192, 46, replace=False)]))
