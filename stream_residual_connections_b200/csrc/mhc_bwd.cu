@@ -64,8 +64,14 @@ __device__ __forceinline__ void store8<float>(float* p, const float (&v)[8]) {
 }
 
 // ---------------------------------------------------------------- B1
+#ifndef MHC_B1_THREADS
+#define MHC_B1_THREADS 128
+#endif
+constexpr int B1_THREADS = MHC_B1_THREADS;   // small blocks: the per-token serial phases of
+constexpr int B1_WARPS = B1_THREADS / 32;    // several blocks overlap on an SM
+
 template <int N, typename TX>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(B1_THREADS)
 b1_kernel(const TX* __restrict__ X, const TX* __restrict__ F, const TX* __restrict__ dXn,
           const TX* __restrict__ dxin, float a0, float a1, float a2, const float* __restrict__ b,
           int64_t T, int C, int t_iters, const float* __restrict__ uu, const float* __restrict__ rr,
@@ -74,7 +80,7 @@ b1_kernel(const TX* __restrict__ X, const TX* __restrict__ F, const TX* __restri
     using L = WS<N>;
     constexpr int P = L::P, NN = N * N;
     __shared__ float trace[MAX_TITERS + 1][NN];
-    __shared__ float red[8][P];
+    __shared__ float red[B1_WARPS][P];
     __shared__ float hp_s[N], ho_s[N], dot[P];
     const int64_t t = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -137,7 +143,7 @@ b1_kernel(const TX* __restrict__ X, const TX* __restrict__ F, const TX* __restri
 #pragma unroll
     for (int p = 0; p < P; ++p) acc[p] = 0.0f;
     const float* ho = ho_s;
-    for (int c = tid * 8; c < C; c += 256 * 8) {
+    for (int c = tid * 8; c < C; c += B1_THREADS * 8) {
         float g[N][8], x[N][8], f[8], gi[8];
 #pragma unroll
         for (int i = 0; i < N; ++i) {
@@ -175,7 +181,7 @@ b1_kernel(const TX* __restrict__ X, const TX* __restrict__ F, const TX* __restri
     if (tid < P) {
         float v = 0.0f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) v += red[w][tid];
+        for (int w = 0; w < B1_WARPS; ++w) v += red[w][tid];
         dot[tid] = v;
     }
     __syncthreads();
@@ -491,7 +497,7 @@ static mhc_status run(const BwdArgs& a, cudaStream_t s)
                                                                                     : launch_pre_fma(pa, s);
         if (st != MHC_OK) return st;
     }
-    b1_kernel<N, TX><<<dim3(unsigned(a.T)), 256, 0, s>>>(
+    b1_kernel<N, TX><<<dim3(unsigned(a.T)), B1_THREADS, 0, s>>>(
         static_cast<const TX*>(a.X), static_cast<const TX*>(a.F), static_cast<const TX*>(a.dXn),
         static_cast<const TX*>(a.dxin), a.alpha[0], a.alpha[1], a.alpha[2], a.b, a.T, a.C, a.t_iters,
         a.u_scratch, a.r_scratch, ws, static_cast<TX*>(a.dF));
