@@ -37,8 +37,13 @@ def _check_V(Vg, Vr, name="V"):
     (50, 128, (3,), "f32", None),
     (29, 256, (2, 5), "bf16", None),
     (40, 640, (1, 4, 7, 16), "f32", 9),
+    (45, 768, (1, 4, 7, 16), "f32", 9),
+    (70, 1024, (3, 9), "bf16", 33),
+    (20, 512, (16, 16, 16, 16), "bf16", None),
 ])
 def test_conv_gs_matches_oracle(T, C, kappa, dtype, seq):
+    """r = 1..4, kappa up to 16, fp32 and bf16, tiles of 8 tokens with ragged ends,
+    sequence restarts (seq)."""
     inp = synth.xhc_inputs(T, N=4, k=2, m=1, C=C, kappa=kappa, dtype=dtype, seed=500 + T + C)
     ws = [torch.from_numpy(w).cuda() for w in inp["conv_w"]]
     V = M.xhc_conv_gs(dev(inp["F"]), ws, seq_len=seq)
@@ -47,8 +52,9 @@ def test_conv_gs_matches_oracle(T, C, kappa, dtype, seq):
     _check_V(host(V), ref)
 
 
-def test_conv_gs_zero_output_gives_zero_components():
-    T, C = 9, 64
+@pytest.mark.parametrize("C", [64, 256])
+def test_conv_gs_zero_output_gives_zero_components(C):
+    T = 9
     F = torch.zeros((T, C), dtype=torch.bfloat16, device="cuda")
     ws = [torch.randn(k, C, device="cuda") for k in (4, 8, 12)]
     V = M.xhc_conv_gs(F, ws)
