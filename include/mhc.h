@@ -239,11 +239,12 @@ typedef enum {
 } mhc_path;
 
 /*
- * mhc_set_path -- process-wide choice of the projection kernel of mhc_pre and
- * xhc_route (for comparisons and tests; both paths compute the same function).
- * The tensor-core paths (TMA + tcgen05.mma, 8-CTA clusters) serve bf16 X and
- * phi, C % 512 == 0, 1 <= T < 2^31, and n in {2, 3, 4} (mhc_pre) or N in
- * {4, 8, 12, 16} (xhc_route).  Under MHC_PATH_TENSOR a call outside that range
+ * mhc_set_path -- process-wide choice of the projection kernel of mhc_pre,
+ * xhc_route and xhc_sparse_update (for comparisons and tests; both paths
+ * compute the same function).  The tensor-core paths (TMA + tcgen05.mma, 8-CTA
+ * clusters) serve bf16 X and phi, C % 512 == 0, 1 <= T < 2^31, and n in
+ * {2, 3, 4} (mhc_pre), N in {4, 8, 12, 16} (xhc_route), k = 4 with Kr <= 4
+ * (xhc_sparse_update).  Under MHC_PATH_TENSOR a call outside that range
  * returns MHC_ERR_UNSUPPORTED.
  */
 mhc_status mhc_set_path(mhc_path path);

@@ -40,6 +40,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
+#include "tma_host.h"
 
 namespace mhc {
 namespace xrtc {
@@ -447,24 +448,6 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 
 // ------------------------------------------------------------------ host
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
 template <int N>
 static int smem_bytes() { return int(layout_for<N>().total) + 1024; }
 
@@ -495,7 +478,7 @@ static mhc_status launch_n(const RouteArgs& a, cudaStream_t s)
     const int64_t tiles64 = (a.T + MT - 1) / MT;
     const int nclusters = int(tiles64 < max_clusters ? tiles64 : max_clusters);
 
-    EncodeTiledFn enc = encode_fn();
+    EncodeTiledFn enc = encode_tiled_fn();
     if (!enc) {
         set_error("xhc_route (tc): cuTensorMapEncodeTiled unavailable");
         return MHC_ERR_CUDA;

@@ -39,6 +39,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
+#include "tma_host.h"
 
 namespace mhc {
 namespace xutc {
@@ -492,24 +493,6 @@ update_tc_kernel(const __grid_constant__ CUtensorMap tmPhi, bf16_t* X, const flo
 
 // ------------------------------------------------------------------ host
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
 template <int KR>
 static mhc_status launch_kr(const UpdateArgs& a, cudaStream_t s)
 {
@@ -537,7 +520,7 @@ static mhc_status launch_kr(const UpdateArgs& a, cudaStream_t s)
     }
     const int64_t tiles64 = (a.T + MT - 1) / MT;
     const int nclusters = int(tiles64 < max_clusters ? tiles64 : max_clusters);
-    EncodeTiledFn enc = encode_fn();
+    EncodeTiledFn enc = encode_tiled_fn();
     if (!enc) {
         set_error("xhc_sparse_update (tc): cuTensorMapEncodeTiled unavailable");
         return MHC_ERR_CUDA;
