@@ -430,7 +430,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                             o[2 * e + 1] = fmaf(hh, bf16_hi(w4[e]), o[2 * e + 1]);
                         }
                     }
-                    store16<false>(x_in + (t0 + tk[u]) * C + cc[u], o);
+                    store16<true>(x_in + (t0 + tk[u]) * C + cc[u], o);   // streaming: keep L2 for the tiles awaiting their re-read
                 }
             }
             __syncwarp();
