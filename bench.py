@@ -14,7 +14,8 @@ collective is on the data path) and the step time is the maximum over ranks.
              L2, so no flush is needed between steps.
 * e2e        the same metric through the public API with pinned HOST buffers:
              every step copies X and F_out host->device and x_in, the
-             coefficients and X_next device->host.
+             coefficients and X_next device->host, pipelined over token
+             chunks on three streams (copies in, kernels, copies out).
 * roofline   the dominant kernel's algorithmic bytes per launch / its mean
              CUDA-event duration inside the timed region, against the measured
              HBM copy bandwidth.
@@ -324,18 +325,36 @@ def run_ours(args, world, rank, local):
     h2d = Xh.numel() * 2 + Fh.numel() * 2
     d2h = sum(t.numel() * t.element_size() for t in outs_h)
 
+    # the step pipelined over token chunks on three streams: host->device copies of
+    # chunk i+1 and device->host copies of chunk i-1 run while chunk i is mixed
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    bounds = [T * i // args.e2e_chunks for i in range(args.e2e_chunks + 1)]
+    devs = (x_in, Hp, Ho, Hr, Xn)
+
     def e2e_step():
-        X.copy_(Xh, non_blocking=True)
-        F.copy_(Fh, non_blocking=True)
-        step()
-        for h, d in zip(outs_h, (x_in, Hp, Ho, Hr, Xn)):
-            h.copy_(d, non_blocking=True)
+        for c in range(args.e2e_chunks):
+            lo, hi = bounds[c], bounds[c + 1]
+            with torch.cuda.stream(s_in):
+                X[lo:hi].copy_(Xh[lo:hi], non_blocking=True)
+                F[lo:hi].copy_(Fh[lo:hi], non_blocking=True)
+            stream.wait_stream(s_in)
+            M.mhc_pre(X[lo:hi], phi, alpha, b, 20, 1e-6, x_in=x_in[lo:hi], H_pre=Hp[lo:hi], H_post=Ho[lo:hi],
+                      H_res=Hr[lo:hi], stream=stream)
+            M.mhc_post(X[lo:hi], F[lo:hi], Ho[lo:hi], Hr[lo:hi], X_next=Xn[lo:hi], stream=stream)
+            s_out.wait_stream(stream)
+            with torch.cuda.stream(s_out):
+                for h, d in zip(outs_h, devs):
+                    h[lo:hi].copy_(d[lo:hi], non_blocking=True)
+        # the next step's first copies overwrite X and F: after this step's reads
+        s_in.wait_stream(stream)
+        stream.wait_stream(s_out)
 
     e2e_step()
     torch.cuda.synchronize(device)
     barrier(world, device)
     s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s2.record(stream)
+    s_in.wait_stream(stream)
     for _ in range(Ke):
         e2e_step()
     e2.record(stream)
@@ -375,7 +394,7 @@ def run_ours(args, world, rank, local):
             "config": config_dict(world),
             "gpu_launches": 2 * K,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "steps": Ke},
+                    "d2h_bytes_per_step": d2h, "steps": Ke, "pipelined_chunks": args.e2e_chunks},
             "roofline": roof,
             "kernels": kern_rows,
             "mhc_pre_fma_path_ms": fma_ms,
@@ -548,6 +567,8 @@ def main(argv=None):
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--e2e-chunks", type=int, default=8,
+                   help="token chunks the e2e step is pipelined over (copies overlap the kernels)")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--compare-fma", type=int, default=1,
