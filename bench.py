@@ -203,7 +203,8 @@ def run_reference(args, world, rank):
     dt = time.perf_counter() - t0
     value = S * args.steps / dt
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    sample = f"{S} tokens per step of the T=8192, n=4, C=4096 bf16 workload (inputs widened to fp64)"
+    w = WORKLOAD
+    sample = f"{S} tokens per step of the T={w['T']}, n={w['n']}, C={w['C']} bf16 workload (inputs widened to fp64)"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -218,11 +219,13 @@ def run_reference(args, world, rank):
 
 
 def config_dict(N: int) -> dict:
-    return {"workload": "mHC forward sublayer (mhc_pre + mhc_post), T=8192 tokens per GPU, "
-                        "n=4, C=4096, bf16 state, fp32 coefficients, Sinkhorn 20 iterations",
+    w = WORKLOAD
+    return {"workload": f"mHC forward sublayer (mhc_pre + mhc_post), T={w['T']} tokens per GPU, "
+                        f"n={w['n']}, C={w['C']}, bf16 state, fp32 coefficients, Sinkhorn 20 iterations",
             "T_per_gpu": WORKLOAD["T"], "n": WORKLOAD["n"], "C": WORKLOAD["C"], "t_iters": 20,
             "global_tokens": WORKLOAD["T"] * N, "parallelism": f"dp{N} (independent token batches)",
-            "l2": "no flush: inputs larger than L2 (X 256 MiB, F_out 64 MiB, X_next 256 MiB vs 126 MB L2)"}
+            "l2": f"no flush: inputs larger than L2 (X {w['T'] * w['n'] * w['C'] * 2 >> 20} MiB, F_out "
+                  f"{w['T'] * w['C'] * 2 >> 20} MiB, X_next {w['T'] * w['n'] * w['C'] * 2 >> 20} MiB vs 126 MB L2)"}
 
 
 # ------------------------------------------------------------------ ours
@@ -382,7 +385,7 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, S, threads = oracle_sample_rate(inp, seconds=args.cpu_seconds, max_tokens=T)
         cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": f"first {S} tokens of the same T=8192, n=4, C=4096 workload, fp64 oracle "
+               "sample": f"first {S} tokens of the same T={T}, n={n}, C={C} workload, fp64 oracle "
                          f"(mhc_pre + mhc_post), OpenMP over tokens"}
 
     if rank == 0:
@@ -557,7 +560,7 @@ def run_secondary(args, local):
 # kernels, from one --set full capture at T=6144 scaled to T=8192 by the token
 # count (profiles/mhc_pre_tc_T6144_n4_C4096_full.md, mhc_post_...).  Set to
 # None whenever a kernel changes after its capture.
-TRAFFIC = {"mhc_pre": 343.3e6, "mhc_post": 541.4e6}
+TRAFFIC = {"mhc_pre": 331.2e6, "mhc_post": 541.3e6}
 
 
 def main(argv=None):
@@ -576,11 +579,19 @@ def main(argv=None):
     p.add_argument("--profile", action="store_true",
                    help="only warm-up + timed kernel launches (for ncu); no e2e, clocks or oracle")
     p.add_argument("--tokens", type=int, default=None, help="override T (profiling of small cases)")
+    p.add_argument("--n", type=int, default=None, help="override n of the mHC forward (the n sweep)")
+    p.add_argument("--C", type=int, default=None, help="override C of the mHC forward")
     p.add_argument("--workload", choices=("mhc_fwd", "xhc", "mhc_bwd"), default="mhc_fwd",
                    help="mhc_fwd: the benchmark line; xhc / mhc_bwd: timing lines for the other kernels")
     args = p.parse_args(argv)
+    global METRIC
     if args.tokens:
         WORKLOAD["T"] = args.tokens
+    if args.n:
+        WORKLOAD["n"] = args.n
+    if args.C:
+        WORKLOAD["C"] = args.C
+    METRIC = f"mHC fwd tokens/s at n={WORKLOAD['n']},C={WORKLOAD['C']}; achieved HBM GB/s vs B200 peak"
     world, rank, local = dist_env()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

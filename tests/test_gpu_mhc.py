@@ -158,6 +158,35 @@ def test_llm_workload_sampled_tokens():
     assert ((got["H_post"] > 0) & (got["H_post"] < 2)).all()
 
 
+def _run_sampled(inp, toks):
+    """Full-size run on the GPU; the sampled tokens' outputs come back to the host,
+    the structural properties are checked on the device over all tokens."""
+    X, F, phi = dev(inp["X"]), dev(inp["F"]), phi_dev(inp["phi"])
+    b = torch.from_numpy(inp["b"]).cuda()
+    x_in, Hp, Ho, Hr = M.mhc_pre(X, phi, inp["alpha"], b, inp["t_iters"], inp["eps"])
+    Xn = M.mhc_post(X, F, Ho, Hr)
+    torch.cuda.synchronize()
+    assert torch.isfinite(Xn.float()).all() and torch.isfinite(x_in.float()).all()
+    assert (Hr >= 0).all() and ((Hp > 0) & (Hp < 1)).all() and ((Ho > 0) & (Ho < 2)).all()
+    assert (Hr.sum(-1) - 1.0).abs().max().item() <= 2e-6
+    sel = torch.from_numpy(np.asarray(toks)).cuda()
+    return dict(x_in=host(x_in[sel]), H_pre=host(Hp[sel]), H_post=host(Ho[sel]), H_res=host(Hr[sel]),
+                X_next=host(Xn[sel]))
+
+
+@pytest.mark.parametrize("name", ["mhc_wide", "mhc_sweep_n2", "mhc_sweep_n8"])
+def test_wide_and_n_sweep_workloads_sampled(name):
+    """The remaining forward workloads at full size: T=32768, n=4, C=7168 (14 channel
+    blocks per CTA on the tensor-core path), and n = 2 (tensor cores) and n = 8 (CUDA
+    cores) at T=8192, C=4096; 48 sampled tokens compared with the oracle."""
+    inp = synth.mhc_inputs(**synth.WORKLOADS[name])
+    T = inp["T"]
+    rng = np.random.default_rng(5)
+    toks = np.unique(np.concatenate([[0, T - 1], rng.choice(T, 46, replace=False)]))
+    got = _run_sampled(inp, toks)
+    _compare(dict(inp, X=inp["X"][toks], F=inp["F"][toks]), got)
+
+
 @pytest.fixture
 def restore_path():
     yield
