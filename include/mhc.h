@@ -262,8 +262,10 @@ mhc_status mhc_set_wait_limit(long long polls);
  * mhc_sync_status -- wait for `stream`, then report and clear the device-side
  * error word: MHC_ERR_TIMEOUT if a kernel of this library gave up a bounded
  * wait since the last call, MHC_ERR_INVALID_ARG if a kernel met an
- * out-of-range stream index in device data, else MHC_OK (or MHC_ERR_CUDA if
- * the stream itself failed).
+ * out-of-range stream index in device data, MHC_ERR_CUDA if a kernel found
+ * its launch configuration inconsistent (shared memory smaller than its
+ * layout, a tile shape it was not written for) and did no work, else MHC_OK
+ * (or MHC_ERR_CUDA if the stream itself failed).
  */
 mhc_status mhc_sync_status(void* stream);
 

@@ -113,13 +113,14 @@ mhc_status mhc_pre(const void* X, mhc_dtype x_dt, const void* phi, mhc_dtype phi
     PreArgs a{X, x_dt, phi, phi_dt, {alpha[0], alpha[1], alpha[2]}, b, T, n, C, t_iters, eps,
               x_in, H_pre, H_post, H_res};
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const bool tc_ok = pre_tc_supported(a);
-    if (g_pre_path == MHC_PATH_TENSOR && !tc_ok) {
+    const bool tc_ok = pre_tc_supported(a), wide_ok = pre_wide_supported(a);
+    if (g_pre_path == MHC_PATH_TENSOR && !tc_ok && !wide_ok) {
         set_error("%s: the tensor-core path was forced but does not support this call "
-                  "(needs bf16 X and phi, n in {2,3,4}, C %% 512 == 0)", fn);
+                  "(needs bf16 X and phi, n in [2, 8], C %% 512 == 0)", fn);
         return MHC_ERR_UNSUPPORTED;
     }
     if (tc_ok && g_pre_path != MHC_PATH_FMA) return launch_pre_tc(a, s);
+    if (wide_ok && g_pre_path != MHC_PATH_FMA) return launch_pre_wide(a, s);
     return launch_pre_fma(a, s);
 }
 
@@ -363,6 +364,11 @@ mhc_status mhc_sync_status(void* stream)
         if (flag & 1u) {
             set_error("a bounded on-device wait expired (error word 0x%x)", flag);
             return MHC_ERR_TIMEOUT;
+        }
+        if (flag & 4u) {
+            set_error("a kernel's check of its own launch configuration failed; it did no work "
+                      "(error word 0x%x)", flag);
+            return MHC_ERR_CUDA;
         }
         set_error("a kernel met an out-of-range stream index; those tokens were left unchanged "
                   "(error word 0x%x)", flag);

@@ -30,6 +30,8 @@ mhc_status launch_pre_fma(const PreArgs& a, cudaStream_t s);
 // {2, 3, 4}, C % 512 == 0 and phi's per-CTA slice resident in shared memory.
 bool pre_tc_supported(const PreArgs& a);
 mhc_status launch_pre_tc(const PreArgs& a, cudaStream_t s);
+bool pre_wide_supported(const PreArgs& a);                       // n = 5..8 (mhc_pre_wide.cu)
+mhc_status launch_pre_wide(const PreArgs& a, cudaStream_t s);
 
 mhc_status launch_conv_gs(const void* F, mhc_dtype dt, const float* W, const int* kappa, int r,
                           int64_t T, int C, int64_t seq_len, float* V, cudaStream_t s);

@@ -4,6 +4,7 @@
 #include "mhc_post.cu"
 #include "mhc_pre_fma.cu"
 #include "mhc_pre_tc.cu"
+#include "mhc_pre_wide.cu"
 #include "xhc_conv_gs.cu"
 #include "xhc_update.cu"
 #include "xhc_update_tc.cu"

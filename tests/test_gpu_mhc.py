@@ -25,6 +25,7 @@ def _run(inp, phi_dtype=None):
     x_in, Hp, Ho, Hr = M.mhc_pre(X, phi, inp["alpha"], b, inp["t_iters"], inp["eps"])
     Xn = M.mhc_post(X, F, Ho, Hr)
     torch.cuda.synchronize()
+    M.mhc_sync_status()
     return dict(x_in=host(x_in), H_pre=host(Hp), H_post=host(Ho), H_res=host(Hr), X_next=host(Xn))
 
 
@@ -166,6 +167,7 @@ def _run_sampled(inp, toks):
     x_in, Hp, Ho, Hr = M.mhc_pre(X, phi, inp["alpha"], b, inp["t_iters"], inp["eps"])
     Xn = M.mhc_post(X, F, Ho, Hr)
     torch.cuda.synchronize()
+    M.mhc_sync_status()                        # no expired wait, no failed self-check
     assert torch.isfinite(Xn.float()).all() and torch.isfinite(x_in.float()).all()
     assert (Hr >= 0).all() and ((Hp > 0) & (Hp < 1)).all() and ((Ho > 0) & (Ho < 2)).all()
     assert (Hr.sum(-1) - 1.0).abs().max().item() <= 2e-6
@@ -207,8 +209,32 @@ def test_tensor_core_path_shapes(T, n, C, restore_path):
     _compare(inp, _run(inp))
 
 
-def test_tensor_and_fma_paths_agree(restore_path):
-    inp = synth.mhc_inputs(700, 4, 1024, "bf16", seed=21)
+@pytest.mark.parametrize("T,n,C", [(300, 8, 512), (1000, 5, 1024), (129, 6, 512), (77, 7, 1536), (1, 8, 512),
+                                   (2048, 8, 2048)])
+def test_tensor_core_path_n5_to_8(T, n, C, restore_path):
+    """n = 5..8: projection kernel on tensor cores (one stream of a 128-token tile per
+    stage, every stream accumulating into the same P columns) + streaming x_in pass."""
+    M.mhc_set_path(M.MHC_PATH_TENSOR)
+    inp = synth.mhc_inputs(T, n, C, "bf16", seed=450 + T + n + C)
+    _compare(inp, _run(inp))
+
+
+def test_n8_without_h_pre_buffer(restore_path):
+    """No H_pre buffer from the caller: the gates wait in the x_in rows between the
+    projection and the x_in pass; x_in must be the same."""
+    inp = synth.mhc_inputs(200, 8, 512, "bf16", seed=460)
+    got = _run(inp)
+    X, phi = dev(inp["X"]), phi_dev(inp["phi"])
+    b = torch.from_numpy(inp["b"]).cuda()
+    x_in2, Hp2, _, _ = M.mhc_pre(X, phi, inp["alpha"], b, inp["t_iters"], inp["eps"], want_H_pre=False)
+    torch.cuda.synchronize()
+    assert Hp2 is None
+    np.testing.assert_array_equal(host(x_in2), got["x_in"])
+
+
+@pytest.mark.parametrize("n", [4, 8])
+def test_tensor_and_fma_paths_agree(n, restore_path):
+    inp = synth.mhc_inputs(700, n, 1024, "bf16", seed=21)
     M.mhc_set_path(M.MHC_PATH_FMA)
     a = _run(inp)
     M.mhc_set_path(M.MHC_PATH_TENSOR)
