@@ -41,9 +41,11 @@ def lib():
         L.orc_xhc_gs.argtypes = [D, D, i64, i32, i32, i32, D]
         L.orc_xhc_sparse_update.argtypes = [D, D, i32, I32, D, D, D, D, i64, i32, i32, i32,
                                             i32, dbl, D, D]
+        L.orc_hc_coeffs.argtypes = [D, D, D, D, i64, i32, i32, dbl, D, D, D]
+        L.orc_amax_gain.argtypes = [D, i32, i64, i32, D]
         for f in ("orc_sinkhorn", "orc_mhc_coeffs", "orc_mhc_apply_pre", "orc_mhc_post",
                   "orc_mhc_backward", "orc_xhc_route", "orc_xhc_conv", "orc_xhc_gs",
-                  "orc_xhc_sparse_update"):
+                  "orc_xhc_sparse_update", "orc_hc_coeffs", "orc_amax_gain"):
             getattr(L, f).restype = None
         _lib = L
     return _lib
@@ -195,3 +197,36 @@ def xhc_sparse_update(X, V, idx, w, phi_act, alpha_act, b_act, t_iters=20, eps=1
                                 _p(w), _p(phi_act), _p(alpha_act), _p(b_act), T, N, C, k,
                                 t_iters, eps, _p(Hr), _p(Ho))
     return Xd, Hr, Ho
+
+
+# ----------------------------------------------------------------- HC (tanh)
+def hc_coeffs(X, theta, alpha, b, eps=1e-6):
+    """Eq.(5) of the mHC paper (the HC parameterisation): per-stream RMSNorm,
+    tanh of the projections, gate factor, static bias.  theta [n+2][C] (rows pre,
+    post, res_0..res_{n-1}); b [n*n+2n].  Returns dict H_pre [T][n], H_post [T][n],
+    H_res [T][n][n]."""
+    X, theta, alpha, b = _c(X), _c(theta), _c(alpha), _c(b)
+    T, n, C = X.shape
+    assert theta.shape == (n + 2, C) and b.shape == (n * n + 2 * n,) and alpha.shape == (3,)
+    Hp = np.empty((T, n)); Ho = np.empty((T, n)); Hr = np.empty((T, n, n))
+    lib().orc_hc_coeffs(_p(X), _p(theta), _p(alpha), _p(b), T, n, C, eps, _p(Hp), _p(Ho), _p(Hr))
+    return dict(H_pre=Hp, H_post=Ho, H_res=Hr)
+
+
+def hc_pre(X, theta, alpha, b, eps=1e-6):
+    """HC coefficients (Eq.5) and x_in = H_pre X (the F_pre input of Eq.3)."""
+    co = hc_coeffs(X, theta, alpha, b, eps)
+    co["x_in"] = mhc_apply_pre(X, co["H_pre"])
+    return co
+
+
+def amax_gain(H_res):
+    """Amax Gain Magnitude (mHC paper section 3.1) of the composite maps
+    M_d = H_res[d-1] ... H_res[0], d = 1..L, per token: H_res [L][T][n][n] ->
+    gain [L][T][2] = (max_i |row sum i|, max_j |column sum j|)."""
+    H = _c(H_res)
+    Lz, T, n, n2 = H.shape
+    assert n == n2 and n <= 8
+    g = np.empty((Lz, T, 2))
+    lib().orc_amax_gain(_p(H), Lz, T, n, _p(g))
+    return g

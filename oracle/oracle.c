@@ -141,6 +141,92 @@ void orc_mhc_post(const double* X, const double* F, const double* H_post,
             }
 }
 
+/* ------------------------------------------------------ HC (tanh) variant */
+
+/* Hyper-Connections coefficients, mHC paper section 3, Eq.(5), for T tokens.
+ * RMSNorm acts on the last dimension: every stream b of X_t is normalised on its
+ * own, x~_b = x_b / sqrt(mean_c x_b[c]^2 + eps) (no weight: it folds into theta).
+ * The dynamic maps are linear projections of x~ followed by tanh, scaled by the
+ * gate factor and shifted by the static map:
+ *   H_pre[b]     = alpha[0] * tanh(theta_pre  . x~_b) + b_pre[b]
+ *   H_post[b]    = alpha[1] * tanh(theta_post . x~_b) + b_post[b]
+ *   H_res[a][b]  = alpha[2] * tanh(theta_res[a] . x~_b) + b_res[a][b]
+ * (theta_res x~^T is n x n with entry [a][b] = theta_res[a] . x~_b).
+ * X [T][n][C]; theta [n+2][C], rows pre, post, res_0 .. res_{n-1};
+ * b [n*n + 2n] = b_pre | b_post | b_res (row-major); alpha[3] = (pre, post, res).
+ * Outputs (nullable): H_pre [T][n], H_post [T][n], H_res [T][n][n]. */
+void orc_hc_coeffs(const double* X, const double* theta, const double* alpha,
+                   const double* b, int64_t T, int n, int C, double eps,
+                   double* H_pre, double* H_post, double* H_res)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        double* xn = (double*)malloc(sizeof(double) * (size_t)n * C);
+        for (int s = 0; s < n; ++s) {                /* RMSNorm per stream */
+            const double* x = X + (t * n + s) * (int64_t)C;
+            double ss = 0.0;
+            for (int c = 0; c < C; ++c) ss += x[c] * x[c];
+            const double r = sqrt(ss / (double)C + eps);
+            for (int c = 0; c < C; ++c) xn[(size_t)s * C + c] = x[c] / r;
+        }
+        for (int s = 0; s < n; ++s) {
+            const double* xs = xn + (size_t)s * C;
+            double proj[2 + 8];                      /* theta_q . x~_s, q = pre, post, res_0.. */
+            for (int q = 0; q < n + 2; ++q) {
+                double acc = 0.0;
+                for (int c = 0; c < C; ++c) acc += theta[(size_t)q * C + c] * xs[c];
+                proj[q] = acc;
+            }
+            if (H_pre) H_pre[t * n + s] = alpha[0] * tanh(proj[0]) + b[s];
+            if (H_post) H_post[t * n + s] = alpha[1] * tanh(proj[1]) + b[n + s];
+            if (H_res)
+                for (int a = 0; a < n; ++a)
+                    H_res[(t * n + a) * n + s] = alpha[2] * tanh(proj[2 + a]) + b[2 * n + a * n + s];
+        }
+        free(xn);
+    }
+}
+
+/* Amax Gain Magnitude, mHC paper section 3.1, of the composite residual map of
+ * Eq.(4).  For every token, the map from the input of layer 0 to the output of
+ * layer d-1 is M_d = H_res[d-1] H_res[d-2] ... H_res[0] (x_d = M_d x_0 + terms of
+ * the layer outputs).  The forward gain is the largest absolute row sum of M_d,
+ * max_i |sum_j M_d[i][j]|; the backward gain the largest absolute column sum,
+ * max_j |sum_i M_d[i][j]|.  H_res [L][T][n][n] (layer-major); gain [L][T][2] =
+ * (forward, backward) for d = 1 .. L. */
+void orc_amax_gain(const double* H_res, int L, int64_t T, int n, double* gain)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        double M[64], P[64];
+        for (int i = 0; i < n; ++i)
+            for (int j = 0; j < n; ++j) M[i * n + j] = i == j ? 1.0 : 0.0;
+        for (int l = 0; l < L; ++l) {
+            const double* H = H_res + ((int64_t)l * T + t) * n * n;
+            for (int i = 0; i < n; ++i)              /* M <- H_res[l] M */
+                for (int j = 0; j < n; ++j) {
+                    double acc = 0.0;
+                    for (int k = 0; k < n; ++k) acc += H[i * n + k] * M[k * n + j];
+                    P[i * n + j] = acc;
+                }
+            memcpy(M, P, sizeof(double) * n * n);
+            double fwd = 0.0, bwd = 0.0;
+            for (int i = 0; i < n; ++i) {
+                double rs = 0.0;
+                for (int j = 0; j < n; ++j) rs += M[i * n + j];
+                if (fabs(rs) > fwd) fwd = fabs(rs);
+            }
+            for (int j = 0; j < n; ++j) {
+                double cs = 0.0;
+                for (int i = 0; i < n; ++i) cs += M[i * n + j];
+                if (fabs(cs) > bwd) bwd = fabs(cs);
+            }
+            gain[((int64_t)l * T + t) * 2 + 0] = fwd;
+            gain[((int64_t)l * T + t) * 2 + 1] = bwd;
+        }
+    }
+}
+
 /* ----------------------------------------------------------- mHC backward */
 
 /* Reverse mode of orc_mhc_coeffs + orc_mhc_apply_pre + orc_mhc_post for T

@@ -129,6 +129,31 @@ def xhc_inputs(T: int, N: int = 16, k: int = 4, m: int = 2, C: int = 2048,
                 Kr=Kr, dtype=dtype, t_iters=20, eps=1e-6, seed=seed)
 
 
+def hc_inputs(T: int, n: int, C: int, dtype: str = "bf16", seed: int = 5,
+              alpha: float = 0.01) -> dict:
+    """Inputs of one HC sublayer (the tanh parameterisation, the mHC paper's Eq. 5,
+    applied by Eq. 3).
+
+    Draw order: X ~ N(0,1) [T][n][C]; F_out ~ N(0,1) [T][C];
+    theta ~ N(0, 1/C) [n+2][C] (rows pre, post, res_0..res_{n-1});
+    b_pre ~ N(0, 0.1) [n]; b_post ~ N(0, 0.1) [n]; the noise of b_res = I_n + N(0, 0.1)
+    [n][n] (the static residual map starts near the identity).  X, F_out and theta
+    take the storage dtype; alpha (all three = ``alpha``) and b are float32.
+    """
+    assert dtype in ("bf16", "f32")
+    rng = np.random.Generator(np.random.PCG64(seed))
+    X = _normal(rng, (T, n, C), 1.0, dtype)
+    F = _normal(rng, (T, C), 1.0, dtype)
+    theta = _normal(rng, (n + 2, C), float(1.0 / np.sqrt(C)), dtype)
+    sd = np.float32(np.sqrt(0.1))
+    b_pre = rng.standard_normal(n, dtype=np.float32) * sd
+    b_post = rng.standard_normal(n, dtype=np.float32) * sd
+    b_res = rng.standard_normal((n, n), dtype=np.float32) * sd + np.eye(n, dtype=np.float32)
+    b = np.concatenate([b_pre, b_post, b_res.reshape(-1)]).astype(np.float32)
+    return dict(X=X, F=F, theta=theta, alpha=np.full(3, alpha, dtype=np.float32), b=b,
+                T=T, n=n, C=C, dtype=dtype, eps=1e-6, seed=seed)
+
+
 def redraw_rows(X: np.ndarray, rows, seed: int, attempt: int, dtype: str) -> None:
     """Replace token rows ``rows`` of a state X [T][N][C] with fresh N(0,1)
     draws from the derived seed (seed, attempt, row) -- used to move routed
@@ -147,4 +172,5 @@ WORKLOADS = {
     "mhc_sweep_n8": dict(T=8192, n=8, C=4096, dtype="bf16", seed=2),
     "xhc": dict(T=8192, N=16, k=4, m=2, C=2048, dtype="bf16", seed=3),
     "mhc_bwd": dict(T=8192, n=4, C=4096, dtype="bf16", seed=4),
+    "hc_llm": dict(T=8192, n=4, C=4096, dtype="bf16", seed=5),
 }
