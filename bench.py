@@ -431,9 +431,22 @@ def mhc_bwd_bytes(T: int, n: int, C: int) -> int:
     return T * (n * C * 2 * 3 + C * 2 * 2) + n * C * P * (2 + 4)
 
 
+def hc_bytes(T: int, n: int, C: int) -> dict:
+    """Bytes per call: hc_pre reads X and theta once and writes x_in and the
+    coefficients; mhc_post as in the mHC step."""
+    return {"hc_pre": T * n * C * 2 + (n + 2) * C * 2 + T * C * 2 + T * (2 * n + n * n) * 4,
+            "mhc_post": T * (2 * (2 * n * C + C) + 4 * (n + n * n))}
+
+
+def amax_bytes(L: int, T: int, n: int) -> int:
+    """Bytes per call: the L x T matrices read once, the per-token gains written once."""
+    return L * T * (n * n * 4 + 2 * 4) + L * 2 * 4
+
+
 def run_secondary(args, local):
-    """Timing lines for the other kernels of the method (xHC sublayer, mHC backward)
-    on their own workloads; one JSON line, rank 0 of a single process."""
+    """Timing lines for the other kernels of the method (xHC sublayer, mHC backward,
+    HC sublayer, Amax Gain diagnostic) on their own workloads; one JSON line, rank 0
+    of a single process."""
     import torch
     import synth
     import stream_residual_connections_b200 as M
@@ -481,6 +494,46 @@ def run_secondary(args, local):
         nbytes = xhc_bytes(T, N, k, m, C, r, sum(inp["kappa"]))
         desc = (f"xHC sublayer (xhc_route + xhc_conv_gs + xhc_sparse_update, X updated in place), T={T}, "
                 f"N={N}, k={k}, m={m}, C={C}, kappa={list(inp['kappa'])}, bf16 state, Sinkhorn 20 iterations")
+    elif args.workload == "hc":
+        wl = dict(synth.WORKLOADS["hc_llm"])
+        if args.tokens:
+            wl["T"] = args.tokens
+        inp = synth.hc_inputs(**wl)
+        T, n, C = inp["T"], inp["n"], inp["C"]
+        X, F = to_dev(inp["X"]), to_dev(inp["F"])
+        theta = to_dev(inp["theta"])
+        b = to_dev(inp["b"])
+        x_in = torch.empty((T, C), dtype=X.dtype, device=device)
+        Hp = torch.empty((T, n), device=device)
+        Ho = torch.empty((T, n), device=device)
+        Hr = torch.empty((T, n, n), device=device)
+        Xn = torch.empty_like(X)
+        names = ("hc_pre", "mhc_post")
+
+        def launches():
+            yield lambda: M.hc_pre(X, theta, inp["alpha"], b, inp["eps"], x_in=x_in, H_pre=Hp, H_post=Ho,
+                                   H_res=Hr, stream=stream)
+            yield lambda: M.mhc_post(X, F, Ho, Hr, X_next=Xn, stream=stream)
+        nbytes = hc_bytes(T, n, C)
+        desc = (f"HC sublayer, tanh coefficients (hc_pre + mhc_post), T={T}, n={n}, C={C}, bf16; inputs "
+                f"larger than L2 (X {T * n * C * 2 >> 20} MiB), no flush")
+    elif args.workload == "amax":
+        Lz, T, n = 64, args.tokens or 65536, 4
+        rng = np.random.default_rng(8)
+        Hh = (np.eye(n, dtype=np.float32) + rng.standard_normal((Lz, T, n, n), dtype=np.float32) * np.float32(0.1))
+        H = torch.from_numpy(Hh).to(device)
+        del Hh
+        gain = torch.empty((Lz, T, 2), device=device)
+        gmax = torch.empty((Lz, 2), device=device)
+        names = ("mhc_amax_gain",)
+        inp = {"H": None}
+
+        def launches():
+            yield lambda: M.mhc_amax_gain(H, gain=gain, gain_max=gmax, stream=stream)
+        nbytes = {"mhc_amax_gain": amax_bytes(Lz, T, n)}
+        desc = (f"Amax Gain Magnitude of the composite residual map over a stack of L={Lz} layers, T={T} "
+                f"tokens, n={n}, fp32 H_res = I + N(0, 0.01) ({Lz * T * n * n * 4 >> 20} MiB, larger than L2, "
+                f"no flush); per-token gains and the maxima over tokens written")
     else:
         wl = dict(synth.WORKLOADS["mhc_bwd"])
         if args.tokens:
@@ -513,7 +566,16 @@ def run_secondary(args, local):
     if not args.no_cpu_baseline:
         import oracle
         oracle.lib()
-        if args.workload == "xhc":
+        if args.workload == "hc":
+            def oracle_step(S):
+                co = oracle.hc_pre(inp["X"][:S], inp["theta"], inp["alpha"], inp["b"], inp["eps"])
+                oracle.mhc_post(inp["X"][:S], inp["F"][:S], co["H_post"], co["H_res"])
+            what = "hc_pre + mhc_post"
+        elif args.workload == "amax":
+            def oracle_step(S):
+                oracle.amax_gain(H[:, :S].cpu().numpy())
+            what = "mhc_amax_gain, L=64"
+        elif args.workload == "xhc":
             def oracle_step(S):
                 rt = oracle.xhc_route(inp["X"][:S], inp["phi_read"], inp["alpha_read"], inp["b_read"], k, m,
                                       inp["eps"])
@@ -581,7 +643,7 @@ def main(argv=None):
     p.add_argument("--tokens", type=int, default=None, help="override T (profiling of small cases)")
     p.add_argument("--n", type=int, default=None, help="override n of the mHC forward (the n sweep)")
     p.add_argument("--C", type=int, default=None, help="override C of the mHC forward")
-    p.add_argument("--workload", choices=("mhc_fwd", "xhc", "mhc_bwd"), default="mhc_fwd",
+    p.add_argument("--workload", choices=("mhc_fwd", "xhc", "mhc_bwd", "hc", "amax"), default="mhc_fwd",
                    help="mhc_fwd: the benchmark line; xhc / mhc_bwd: timing lines for the other kernels")
     args = p.parse_args(argv)
     global METRIC

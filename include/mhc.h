@@ -103,6 +103,54 @@ mhc_status mhc_post(const void* X, const void* F_out, mhc_dtype dt, const float*
                     const float* H_res, int64_t T, int n, int C, void* X_next, void* stream);
 
 /*
+ * hc_pre -- the pre half of one sublayer with the HC (tanh) parameterisation,
+ * the unconstrained predecessor of mHC.   [mHC] section 3, Eq.(5) and Eq.(3).
+ * The post half is mhc_post (same Eq.(3)).
+ *
+ * For every token t and stream s (RMSNorm over the last dimension: each
+ * stream on its own):
+ *   r_s = sqrt(sum_c X_t[s][c]^2 / C + eps);  g_{q,s} = theta[q] . X_t[s] / r_s
+ *   H_pre[s]    = alpha_pre  * tanh(g_{0,s})   + b[s]
+ *   H_post[s]   = alpha_post * tanh(g_{1,s})   + b[n + s]
+ *   H_res[a][s] = alpha_res  * tanh(g_{2+a,s}) + b[2n + a*n + s]
+ *   x_in[c] = sum_s H_pre[s] * X_t[s][c]
+ *
+ *   X      [T][n][C], dtype x_dt                        (read)
+ *   theta  [n+2][C], dtype theta_dt: rows theta_pre, theta_post, theta_res[0..n-1] (read)
+ *   alpha  HOST float[3] = (alpha_pre, alpha_post, alpha_res)
+ *   b      [n*n + 2n] fp32 = b_pre | b_post | b_res (row-major)   (read)
+ *   x_in   [T][C], dtype x_dt (written); H_pre [T][n] fp32, may be NULL;
+ *   H_post [T][n] fp32; H_res [T][n][n] fp32 (H_res[t][a][s] weights source
+ *   stream s into a) (written).
+ * Supported (x_dt, theta_dt): (F32, F32), (BF16, BF16), (BF16, F32).  Outputs
+ * must not overlap any input.  Errors as mhc_pre.
+ */
+mhc_status hc_pre(const void* X, mhc_dtype x_dt, const void* theta, mhc_dtype theta_dt,
+                  const float* alpha, const float* b, int64_t T, int n, int C, float eps,
+                  void* x_in, float* H_pre, float* H_post, float* H_res, void* stream);
+
+/*
+ * mhc_amax_gain -- the Amax Gain Magnitude of the composite residual map of a
+ * stack of L layers.   [mHC] section 3 Eq.(4) and section 3.1.
+ *
+ * For every token t and depth d = 1..L, with M_d = H_res[d-1] ... H_res[0]
+ * (newest layer on the left; x_d = M_d x_0 + terms of the layer outputs):
+ *   forward gain  = max_i |sum_j M_d[i][j]|      (largest absolute row sum)
+ *   backward gain = max_j |sum_i M_d[i][j]|      (largest absolute column sum)
+ * products and sums in fp32.
+ *
+ *   H_res    [L][T][n][n] fp32, layer-major (e.g. the H_res of L mhc_pre or
+ *            hc_pre calls stacked) (read)
+ *   gain     [L][T][2] fp32 = (forward, backward), may be NULL (written)
+ *   gain_max [L][2] fp32, the maxima over the tokens, may be NULL (written;
+ *            zeroed by this call on `stream` first)
+ * At least one output must be given; pointers 16-byte aligned; a NaN product
+ * is skipped by the maxima.  n in [1, 8]; L, T >= 0.
+ */
+mhc_status mhc_amax_gain(const float* H_res, int L, int64_t T, int n, float* gain,
+                         float* gain_max, void* stream);
+
+/*
  * xhc_route -- stream routing and dense read of one xHC sublayer.
  * [xHC] "sparse residual stream architecture", steps 1 (routing: m fixed
  * streams with weight 1, k-m chosen by TopK over sigmoid scores derived from

@@ -1,5 +1,6 @@
 """B200 (sm_100a) residual-stream mixing: mHC pre/post, xHC routing / conv +
-Gram-Schmidt / sparse update, and the mHC backward.
+Gram-Schmidt / sparse update, the mHC backward, and the HC (tanh) pre half with
+the Amax Gain diagnostic.
 
 This module is a thin binding over the C ABI of ``libmhc.so`` (declared in
 ``include/mhc.h``): it checks tensor devices, dtypes and contiguity, allocates
@@ -57,9 +58,11 @@ def _load():
     L.xhc_sparse_update.argtypes = [vp, i32, vp, i32, vp, vp, vp, fp, vp, i64, i32, i32, i32, i32,
                                     f32, vp, vp, vp]
     L.mhc_set_wait_limit.argtypes = [ct.c_longlong]
+    L.hc_pre.argtypes = [vp, i32, vp, i32, fp, vp, i64, i32, i32, f32, vp, vp, vp, vp, vp]
+    L.mhc_amax_gain.argtypes = [vp, i32, i64, i32, vp, vp, vp]
     for name in ("mhc_pre", "mhc_post", "mhc_sync_status", "mhc_set_path", "mhc_set_wait_limit",
                  "xhc_conv_gs", "xhc_sparse_update", "xhc_route", "mhc_backward",
-                 "mhc_backward_noalloc"):
+                 "mhc_backward_noalloc", "hc_pre", "mhc_amax_gain"):
         getattr(L, name).restype = ct.c_int
     return L
 
@@ -130,6 +133,42 @@ def mhc_pre(X, phi, alpha, b, t_iters: int = 20, eps: float = 1e-6, *, x_in=None
                        int(t_iters), float(eps), _ptr(x_in), _ptr(H_pre), _ptr(H_post),
                        _ptr(H_res), _stream(stream)))
     return x_in, H_pre, H_post, H_res
+
+
+def hc_pre(X, theta, alpha, b, eps: float = 1e-6, *, x_in=None, H_pre=None, H_post=None, H_res=None,
+           want_H_pre: bool = True, stream=None):
+    """Pre half of one sublayer with the HC (tanh) coefficients (see include/mhc.h).
+    X [T][n][C], theta [n+2][C] (rows pre, post, res_0..res_{n-1}), alpha: 3 host
+    floats, b [n^2+2n] fp32.  Returns (x_in, H_pre, H_post, H_res); the post half is
+    mhc_post."""
+    T, n, C = X.shape
+    dev = X.device
+    if x_in is None:
+        x_in = torch.empty((T, C), dtype=X.dtype, device=dev)
+    if H_pre is None and want_H_pre:
+        H_pre = torch.empty((T, n), dtype=torch.float32, device=dev)
+    if H_post is None:
+        H_post = torch.empty((T, n), dtype=torch.float32, device=dev)
+    if H_res is None:
+        H_res = torch.empty((T, n, n), dtype=torch.float32, device=dev)
+    _check(native().hc_pre(_ptr(X), _dt(X), _ptr(theta), _dt(theta), _host3(alpha), _ptr(b), T, n, C,
+                           float(eps), _ptr(x_in), _ptr(H_pre), _ptr(H_post), _ptr(H_res), _stream(stream)))
+    return x_in, H_pre, H_post, H_res
+
+
+def mhc_amax_gain(H_res, *, gain=None, gain_max=None, want_gain: bool = True, stream=None):
+    """Amax Gain Magnitude of the composite maps H_res[d-1]..H_res[0], d = 1..L (see
+    include/mhc.h).  H_res [L][T][n][n] fp32.  Returns (gain [L][T][2] or None,
+    gain_max [L][2]): (forward, backward) = largest absolute row / column sum."""
+    Lz, T, n, n2 = H_res.shape
+    if n != n2 or H_res.dtype != torch.float32:
+        raise ValueError("H_res must be fp32 [L][T][n][n]")
+    if gain is None and want_gain:
+        gain = torch.empty((Lz, T, 2), dtype=torch.float32, device=H_res.device)
+    if gain_max is None:
+        gain_max = torch.empty((Lz, 2), dtype=torch.float32, device=H_res.device)
+    _check(native().mhc_amax_gain(_ptr(H_res), Lz, T, n, _ptr(gain), _ptr(gain_max), _stream(stream)))
+    return gain, gain_max
 
 
 def mhc_post(X, F_out, H_post, H_res, *, X_next=None, stream=None):

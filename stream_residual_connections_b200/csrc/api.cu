@@ -72,7 +72,7 @@ extern "C" {
 
 const char* mhc_last_error(void) { return g_msg; }
 
-int mhc_version(void) { return 100; }
+int mhc_version(void) { return 101; }
 
 mhc_status mhc_pre(const void* X, mhc_dtype x_dt, const void* phi, mhc_dtype phi_dt,
                    const float* alpha, const float* b, int64_t T, int n, int C, int t_iters,
@@ -148,6 +148,68 @@ mhc_status mhc_post(const void* X, const void* F_out, mhc_dtype dt, const float*
                 !overlap(rXn, range_of(H_res, size_t(T) * n * n * 4)),
             MHC_ERR_INVALID_ARG, "%s: X_next overlaps F_out or a coefficient array", fn);
     return launch_post(X, F_out, dt, H_post, H_res, T, n, C, X_next, static_cast<cudaStream_t>(stream));
+}
+
+mhc_status hc_pre(const void* X, mhc_dtype x_dt, const void* theta, mhc_dtype theta_dt, const float* alpha,
+                  const float* b, int64_t T, int n, int C, float eps, void* x_in, float* H_pre, float* H_post,
+                  float* H_res, void* stream)
+{
+    const char* fn = "hc_pre";
+    g_msg[0] = 0;
+    REQUIRE(valid_dt(x_dt) && valid_dt(theta_dt), MHC_ERR_INVALID_ARG, "%s: unknown dtype", fn);
+    REQUIRE(n >= 1 && n <= 8, MHC_ERR_INVALID_ARG, "%s: n=%d outside [1, 8]", fn, n);
+    REQUIRE(C > 0 && C % 8 == 0, MHC_ERR_INVALID_ARG, "%s: C=%d must be a positive multiple of 8", fn, C);
+    REQUIRE(T >= 0, MHC_ERR_INVALID_ARG, "%s: T=%lld < 0", fn, (long long)T);
+    REQUIRE(eps >= 0.0f, MHC_ERR_INVALID_ARG, "%s: eps < 0", fn);
+    REQUIRE(alpha != nullptr, MHC_ERR_INVALID_ARG, "%s: alpha (host float[3]) is NULL", fn);
+    REQUIRE(!(x_dt == MHC_F32 && theta_dt == MHC_BF16), MHC_ERR_UNSUPPORTED,
+            "%s: fp32 X with bf16 theta is not supported", fn);
+    if (T == 0) return MHC_OK;
+    REQUIRE_PTR(X, "X");
+    REQUIRE_PTR(theta, "theta");
+    REQUIRE_PTR(b, "b");
+    REQUIRE_PTR(x_in, "x_in");
+    REQUIRE_PTR(H_post, "H_post");
+    REQUIRE_PTR(H_res, "H_res");
+    if (H_pre) REQUIRE(aligned16(H_pre), MHC_ERR_INVALID_ARG, "%s: H_pre is not 16-byte aligned", fn);
+    const int P = n * n + 2 * n;
+    const size_t es = dt_size(x_dt);
+    const Range rX = range_of(X, size_t(T) * n * C * es), rth = range_of(theta, size_t(n + 2) * C * dt_size(theta_dt)),
+                rb = range_of(b, size_t(P) * 4);
+    const Range outs[4] = {range_of(x_in, size_t(T) * C * es), range_of(H_pre, H_pre ? size_t(T) * n * 4 : 0),
+                           range_of(H_post, size_t(T) * n * 4), range_of(H_res, size_t(T) * n * n * 4)};
+    for (int i = 0; i < 4; ++i) {
+        REQUIRE(!overlap(outs[i], rX) && !overlap(outs[i], rth) && !overlap(outs[i], rb),
+                MHC_ERR_INVALID_ARG, "%s: an output overlaps an input", fn);
+        for (int j = 0; j < i; ++j)
+            REQUIRE(!overlap(outs[i], outs[j]), MHC_ERR_INVALID_ARG, "%s: outputs overlap", fn);
+    }
+    HcArgs a{X, x_dt, theta, theta_dt, {alpha[0], alpha[1], alpha[2]}, b, T, n, C, eps, x_in, H_pre, H_post, H_res};
+    return launch_hc_pre(a, static_cast<cudaStream_t>(stream));
+}
+
+mhc_status mhc_amax_gain(const float* H_res, int L, int64_t T, int n, float* gain, float* gain_max, void* stream)
+{
+    const char* fn = "mhc_amax_gain";
+    g_msg[0] = 0;
+    REQUIRE(n >= 1 && n <= 8, MHC_ERR_INVALID_ARG, "%s: n=%d outside [1, 8]", fn, n);
+    REQUIRE(L >= 0 && T >= 0, MHC_ERR_INVALID_ARG, "%s: L=%d, T=%lld must be >= 0", fn, L, (long long)T);
+    REQUIRE(gain || gain_max, MHC_ERR_INVALID_ARG, "%s: neither gain nor gain_max given", fn);
+    if (L == 0) return MHC_OK;
+    if (gain_max) REQUIRE(aligned16(gain_max), MHC_ERR_INVALID_ARG, "%s: gain_max is not 16-byte aligned", fn);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (gain_max) {
+        const mhc_status st = cuda_status(cudaMemsetAsync(gain_max, 0, size_t(L) * 2 * 4, s), fn);
+        if (st != MHC_OK) return st;
+    }
+    if (T == 0) return MHC_OK;
+    REQUIRE_PTR(H_res, "H_res");
+    if (gain) REQUIRE(aligned16(gain), MHC_ERR_INVALID_ARG, "%s: gain is not 16-byte aligned", fn);
+    const Range rH = range_of(H_res, size_t(L) * T * n * n * 4);
+    const Range rg = range_of(gain, gain ? size_t(L) * T * 2 * 4 : 0), rm = range_of(gain_max, gain_max ? size_t(L) * 8 : 0);
+    REQUIRE(!overlap(rg, rH) && !overlap(rm, rH) && !overlap(rg, rm), MHC_ERR_INVALID_ARG,
+            "%s: an output overlaps H_res or the other output", fn);
+    return launch_amax_gain(H_res, L, T, n, gain, gain_max, s);
 }
 
 mhc_status xhc_route(const void* X, mhc_dtype dt, const void* phi_read, const float* alpha_read,

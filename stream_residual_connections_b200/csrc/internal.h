@@ -66,6 +66,17 @@ int backward_b3_segments(int64_t T);
 size_t backward_record_stride(int n);            // floats per token record (0: unsupported n)
 mhc_status launch_backward(const BwdArgs& a, cudaStream_t s);
 
+// HC (tanh) coefficients + F_pre input (hc_pre.cu); Amax Gain of a stack of H_res.
+struct HcArgs {
+    const void* X; mhc_dtype x_dt; const void* theta; mhc_dtype t_dt;
+    float alpha[3]; const float* b;
+    int64_t T; int n; int C; float eps;
+    void* x_in; float* H_pre; float* H_post; float* H_res;
+};
+mhc_status launch_hc_pre(const HcArgs& a, cudaStream_t s);
+mhc_status launch_amax_gain(const float* H, int L, int64_t T, int n, float* gain, float* gain_max,
+                            cudaStream_t s);
+
 // Which mhc_pre path to take (MHC_PRE_PATH_*), process-wide.
 extern int g_pre_path;
 
