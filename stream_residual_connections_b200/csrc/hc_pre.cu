@@ -24,9 +24,10 @@
 // The Amax Gain Magnitude ([mHC] section 3.1) of the composite map of Eq.(4),
 // M_d = H_res[d-1] ... H_res[0]: one thread per token carries M (n x n fp32) through
 // the layers, and after each layer writes max_i |row sum i| (forward) and
-// max_j |column sum j| (backward); the maxima over the tokens go through one
-// atomicMax per warp on the bit patterns (non-negative floats order like their
-// bits, so the result does not depend on the order).
+// max_j |column sum j| (backward); the maxima over the tokens are reduced per warp
+// and per block and reach the output through atomicMax on the bit patterns
+// (non-negative floats order like their bits, so the result does not depend on
+// the order).
 #include "common.cuh"
 #include "internal.h"
 
@@ -181,67 +182,90 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 template <int N>
+__device__ __forceinline__ void load_layer(const float* __restrict__ h, float (&Hl)[N * N]) {
+    if constexpr ((N * N) % 4 == 0) {       // a token's n*n floats are 16-byte aligned
+#pragma unroll
+        for (int e = 0; e < N * N; e += 4) {
+            const float4 v = __ldcs(reinterpret_cast<const float4*>(h + e));
+            Hl[e] = v.x; Hl[e + 1] = v.y; Hl[e + 2] = v.z; Hl[e + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < N * N; ++e) Hl[e] = __ldcs(h + e);
+    }
+}
+
+// Persistent blocks walk groups of 256 tokens.  The maxima over tokens are
+// reduced per warp (shuffles), then per block in shared memory (bmax [L][2], when
+// it fits), and each block adds its L x 2 maxima to gmax with one global atomic
+// per entry at the end, instead of one per warp and layer on the same few
+// addresses.
+template <int N>
 __global__ void __launch_bounds__(256)
 amax_gain_kernel(const float* __restrict__ H, int L, int64_t T, float* __restrict__ gain,
-                 unsigned int* __restrict__ gmax)
+                 unsigned int* __restrict__ gmax, int block_max)
 {
-    const int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-    const bool live = t < T;               // idle threads still join the warp maxima
-    float M[N][N];
+    extern __shared__ unsigned int bmax[];
+    const bool use_b = gmax && block_max;
+    if (use_b) {
+        for (int i = threadIdx.x; i < 2 * L; i += blockDim.x) bmax[i] = 0u;
+        __syncthreads();
+    }
+    for (int64_t base = int64_t(blockIdx.x) * blockDim.x; base < T; base += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t t = base + threadIdx.x;
+        const bool live = t < T;           // idle threads still join the warp maxima
+        float M[N][N];
 #pragma unroll
-    for (int i = 0; i < N; ++i)
+        for (int i = 0; i < N; ++i)
 #pragma unroll
-        for (int j = 0; j < N; ++j) M[i][j] = i == j ? 1.0f : 0.0f;
-    for (int l = 0; l < L; ++l) {
-        float fw = 0.0f, bw = 0.0f;
-        if (live) {
-            const float* h = H + (int64_t(l) * T + t) * (N * N);
-            float Hl[N * N];
-            if constexpr ((N * N) % 4 == 0) {   // rows of n*n floats are 16-byte aligned
+            for (int j = 0; j < N; ++j) M[i][j] = i == j ? 1.0f : 0.0f;
+        for (int l = 0; l < L; ++l) {
+            float fw = 0.0f, bw = 0.0f;
+            if (live) {
+                float Hl[N * N];
+                load_layer<N>(H + (int64_t(l) * T + t) * (N * N), Hl);
+                float P[N][N];               // M <- H_res[l] M
 #pragma unroll
-                for (int e = 0; e < N * N; e += 4) {
-                    const float4 v = __ldcs(reinterpret_cast<const float4*>(h + e));
-                    Hl[e] = v.x; Hl[e + 1] = v.y; Hl[e + 2] = v.z; Hl[e + 3] = v.w;
+                for (int i = 0; i < N; ++i)
+#pragma unroll
+                    for (int j = 0; j < N; ++j) {
+                        float acc = 0.0f;
+#pragma unroll
+                        for (int k = 0; k < N; ++k) acc = fmaf(Hl[i * N + k], M[k][j], acc);
+                        P[i][j] = acc;
+                    }
+#pragma unroll
+                for (int i = 0; i < N; ++i)
+#pragma unroll
+                    for (int j = 0; j < N; ++j) M[i][j] = P[i][j];
+#pragma unroll
+                for (int i = 0; i < N; ++i) {
+                    float rs = 0.0f, cs = 0.0f;
+#pragma unroll
+                    for (int j = 0; j < N; ++j) {
+                        rs += M[i][j];
+                        cs += M[j][i];
+                    }
+                    if (fabsf(rs) > fw) fw = fabsf(rs);
+                    if (fabsf(cs) > bw) bw = fabsf(cs);
                 }
-            } else {
-#pragma unroll
-                for (int e = 0; e < N * N; ++e) Hl[e] = __ldcs(h + e);
+                if (gain) *reinterpret_cast<float2*>(gain + (int64_t(l) * T + t) * 2) = make_float2(fw, bw);
             }
-            float P[N][N];                       // M <- H_res[l] M
-#pragma unroll
-            for (int i = 0; i < N; ++i)
-#pragma unroll
-                for (int j = 0; j < N; ++j) {
-                    float acc = 0.0f;
-#pragma unroll
-                    for (int k = 0; k < N; ++k) acc = fmaf(Hl[i * N + k], M[k][j], acc);
-                    P[i][j] = acc;
+            if (gmax) {
+                fw = warp_max(fw);
+                bw = warp_max(bw);
+                if ((threadIdx.x & 31) == 0) {
+                    unsigned int* dst = use_b ? bmax : gmax;
+                    atomicMax(dst + 2 * l, __float_as_uint(fw));
+                    atomicMax(dst + 2 * l + 1, __float_as_uint(bw));
                 }
-#pragma unroll
-            for (int i = 0; i < N; ++i)
-#pragma unroll
-                for (int j = 0; j < N; ++j) M[i][j] = P[i][j];
-#pragma unroll
-            for (int i = 0; i < N; ++i) {
-                float rs = 0.0f, cs = 0.0f;
-#pragma unroll
-                for (int j = 0; j < N; ++j) {
-                    rs += M[i][j];
-                    cs += M[j][i];
-                }
-                if (fabsf(rs) > fw) fw = fabsf(rs);
-                if (fabsf(cs) > bw) bw = fabsf(cs);
             }
-            if (gain) *reinterpret_cast<float2*>(gain + (int64_t(l) * T + t) * 2) = make_float2(fw, bw);
         }
-        if (gmax) {
-            fw = warp_max(fw);
-            bw = warp_max(bw);
-            if ((threadIdx.x & 31) == 0) {
-                atomicMax(gmax + 2 * l, __float_as_uint(fw));
-                atomicMax(gmax + 2 * l + 1, __float_as_uint(bw));
-            }
-        }
+    }
+    if (use_b) {
+        __syncthreads();
+        for (int i = threadIdx.x; i < 2 * L; i += blockDim.x)
+            if (bmax[i]) atomicMax(gmax + i, bmax[i]);
     }
 }
 
@@ -260,10 +284,22 @@ mhc_status launch_amax_gain(const float* H, int L, int64_t T, int n, float* gain
                             cudaStream_t s)
 {
     unsigned int* gm = reinterpret_cast<unsigned int*>(gain_max);
-    const unsigned blocks = unsigned((T + 255) / 256);
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_status(e, "mhc_amax_gain: SM count");
+    }
+    // two resident blocks per SM, each walking groups of 256 tokens; the block
+    // maxima live in shared memory up to L = 6144 layers (48 KB)
+    const int64_t groups = (T + 255) / 256;
+    const unsigned blocks = unsigned(groups < 2 * sms ? groups : 2 * sms);
+    const int block_max = L <= 6144 ? 1 : 0;
+    const size_t shm = gain_max && block_max ? size_t(L) * 2 * 4 : 0;
     switch (n) {
 #define MHC_AMAX_CASE(K) \
-        case K: hc::amax_gain_kernel<K><<<blocks, 256, 0, s>>>(H, L, T, gain, gm); break;
+        case K: hc::amax_gain_kernel<K><<<blocks, 256, shm, s>>>(H, L, T, gain, gm, block_max); break;
         MHC_AMAX_CASE(1) MHC_AMAX_CASE(2) MHC_AMAX_CASE(3) MHC_AMAX_CASE(4)
         MHC_AMAX_CASE(5) MHC_AMAX_CASE(6) MHC_AMAX_CASE(7) MHC_AMAX_CASE(8)
 #undef MHC_AMAX_CASE

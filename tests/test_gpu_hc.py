@@ -103,24 +103,33 @@ def test_hc_llm_workload_sampled_tokens():
 # ------------------------------------------------------------------ Amax Gain
 
 def _gain_tolerance(H: np.ndarray) -> np.ndarray:
-    """Bound of the fp32 error of the gains: per depth d, every product and sum adds
-    at most a few ulps of the absolute composite, |M_d| <= |H_(d-1)| ... |H_0|
-    entrywise; 4 n d 2^-24 times its largest absolute row / column sum."""
+    """First-order bound of the fp32 error of the gains: a rounding error made at
+    depth k travels to depth d through the same maps as M itself, so each of the
+    about n d roundings up to depth d adds at most a few ulps of |M_d| (the
+    composite of the same fp32 matrices, in fp64): 4 n d 2^-24 times its largest
+    absolute row / column sum (|sum_j M[i][j]| <= sum_j |M[i][j]|).  Deep random
+    chains measured at under 1/30 of it."""
     Lz, T, n, _ = H.shape
-    A = np.broadcast_to(np.eye(n), (T, n, n)).copy()
+    Mc = np.broadcast_to(np.eye(n), (T, n, n)).copy()
     tol = np.empty((Lz, T, 2))
     for d in range(Lz):
-        A = np.abs(H[d]) @ A
+        Mc = np.einsum("tik,tkj->tij", H[d], Mc)
+        A = np.abs(Mc)
         tol[d, :, 0] = A.sum(2).max(1)
         tol[d, :, 1] = A.sum(1).max(1)
         tol[d] *= 4 * n * (d + 1) * 2.0 ** -24
     return tol + 1e-30
 
 
-@pytest.mark.parametrize("Lz,T,n", [(24, 1000, 4), (5, 300, 1), (9, 257, 3), (12, 64, 8), (1, 1, 2)])
+@pytest.mark.parametrize("Lz,T,n", [(24, 1000, 4), (5, 300, 1), (9, 257, 3), (12, 64, 8), (1, 1, 2),
+                                    (2, 80000, 2), (6200, 40, 2)])
 def test_amax_gain_matches_oracle(Lz, T, n):
+    """Includes more token groups than resident blocks (T = 80000: every block walks
+    several groups) and more layers than the block maxima's shared memory holds
+    (L = 6200: maxima straight to global memory)."""
     rng = np.random.default_rng(600 + Lz + T + n)
-    H = (np.eye(n) + rng.normal(size=(Lz, T, n, n)) * 0.3).astype(np.float32)
+    sd = 0.3 if Lz <= 64 else 0.3 * np.sqrt(24 / Lz)   # deep stacks: keep the product finite
+    H = (np.eye(n) + rng.normal(size=(Lz, T, n, n)) * sd).astype(np.float32)
     g, gm = M.mhc_amax_gain(torch.from_numpy(H).cuda())
     torch.cuda.synchronize()
     g, gm = host(g), host(gm)
