@@ -517,6 +517,36 @@ def run_secondary(args, local):
         nbytes = hc_bytes(T, n, C)
         desc = (f"HC sublayer, tanh coefficients (hc_pre + mhc_post), T={T}, n={n}, C={C}, bf16; inputs "
                 f"larger than L2 (X {T * n * C * 2 >> 20} MiB), no flush")
+    elif args.workload == "mhc_tf32":
+        wl = dict(synth.WORKLOADS["mhc_llm"])
+        if args.tokens:
+            wl["T"] = args.tokens
+        inp = synth.mhc_inputs(**wl, phi_dtype="tf32")
+        T, n, C = inp["T"], inp["n"], inp["C"]
+        X, F = to_dev(inp["X"]), to_dev(inp["F"])
+        phiT = to_dev(np.ascontiguousarray(inp["phi"].T))
+        pair = M.mhc_phi_tf32_pair(phiT, n, stream=stream)      # once per update of phi
+        b = to_dev(inp["b"])
+        x_in = torch.empty((T, C), dtype=X.dtype, device=device)
+        Hp = torch.empty((T, n), device=device)
+        Ho = torch.empty((T, n), device=device)
+        Hr = torch.empty((T, n, n), device=device)
+        Xn = torch.empty_like(X)
+        names = ("mhc_pre", "mhc_post", "mhc_phi_tf32_pair")
+
+        def launches():
+            yield lambda: M.mhc_pre(X, pair, inp["alpha"], b, 20, 1e-6, x_in=x_in, H_pre=Hp, H_post=Ho, H_res=Hr,
+                                    phi_tf32_pair=True, stream=stream)
+            yield lambda: M.mhc_post(X, F, Ho, Hr, X_next=Xn, stream=stream)
+            yield lambda: M.mhc_phi_tf32_pair(phiT, n, pair=pair, stream=stream)
+        P = n * n + 2 * n
+        RH = (P + 15) // 16 * 16
+        pre_b = T * (2 * n * C + 2 * C + 4 * (2 * n + n * n)) + 2 * RH * n * C * 2
+        nbytes = {"mhc_pre": pre_b, "mhc_post": T * (2 * (2 * n * C + C) + 4 * (n + n * n)),
+                  "mhc_phi_tf32_pair": P * n * C * 4 + 2 * RH * n * C * 2}
+        desc = (f"mHC forward sublayer with phi in tf32 (the pages' Eq.10 dtype; bf16 pair on tensor cores), "
+                f"T={T}, n={n}, C={C}, bf16 state; the pair packing (once per phi update) is timed as a "
+                f"third kernel of the loop")
     elif args.workload == "amax":
         Lz, T, n = 64, args.tokens or 65536, 4
         rng = np.random.default_rng(8)
@@ -566,7 +596,11 @@ def run_secondary(args, local):
     if not args.no_cpu_baseline:
         import oracle
         oracle.lib()
-        if args.workload == "hc":
+        if args.workload == "mhc_tf32":
+            def oracle_step(S):
+                oracle.mhc_forward(inp["X"][:S], inp["F"][:S], inp["phi"], inp["alpha"], inp["b"], 20, 1e-6)
+            what = "mhc_pre + mhc_post, tf32 phi"
+        elif args.workload == "hc":
             def oracle_step(S):
                 co = oracle.hc_pre(inp["X"][:S], inp["theta"], inp["alpha"], inp["b"], inp["eps"])
                 oracle.mhc_post(inp["X"][:S], inp["F"][:S], co["H_post"], co["H_res"])
@@ -643,7 +677,7 @@ def main(argv=None):
     p.add_argument("--tokens", type=int, default=None, help="override T (profiling of small cases)")
     p.add_argument("--n", type=int, default=None, help="override n of the mHC forward (the n sweep)")
     p.add_argument("--C", type=int, default=None, help="override C of the mHC forward")
-    p.add_argument("--workload", choices=("mhc_fwd", "xhc", "mhc_bwd", "hc", "amax"), default="mhc_fwd",
+    p.add_argument("--workload", choices=("mhc_fwd", "xhc", "mhc_bwd", "hc", "amax", "mhc_tf32"), default="mhc_fwd",
                    help="mhc_fwd: the benchmark line; xhc / mhc_bwd: timing lines for the other kernels")
     args = p.parse_args(argv)
     global METRIC

@@ -48,7 +48,9 @@ typedef enum {
     MHC_ERR_TIMEOUT = 4       /* a bounded on-device wait expired (see mhc_sync_status)*/
 } mhc_status;
 
-typedef enum { MHC_F32 = 0, MHC_BF16 = 1 } mhc_dtype;
+/* MHC_TF32_PAIR: only as the phi dtype of mhc_pre -- a tf32 projection matrix
+ * ([mHC] Eq.(10)) in the exact bf16 pair layout written by mhc_phi_tf32_pair. */
+typedef enum { MHC_F32 = 0, MHC_BF16 = 1, MHC_TF32_PAIR = 2 } mhc_dtype;
 
 /* Message of the last failing call on this thread ("" if none).  Never NULL. */
 const char* mhc_last_error(void);
@@ -79,13 +81,36 @@ int mhc_version(void);
  *   H_pre  [T][n] fp32, may be NULL                    (written)
  *   H_post [T][n] fp32                                 (written)
  *   H_res  [T][n][n] fp32 (H_res[t][i][j] weights source stream j into i) (written)
- * Supported (x_dt, phi_dt): (F32, F32), (BF16, BF16), (BF16, F32).
+ * Supported (x_dt, phi_dt): (F32, F32), (BF16, BF16), (BF16, F32), and
+ * (BF16, TF32_PAIR): phi is then the [2*RH][n*C] bf16 pair of a tf32 phi^T
+ * from mhc_phi_tf32_pair (the pages' Eq.(10)-(11) dtypes), and the
+ * projection is x . (hi + lo) = x . phi_tf32 with fp32 accumulation.
  * Outputs must not overlap any input.
  */
 mhc_status mhc_pre(const void* X, mhc_dtype x_dt, const void* phi, mhc_dtype phi_dt,
                    const float* alpha, const float* b, int64_t T, int n, int C,
                    int t_iters, float eps, void* x_in, float* H_pre, float* H_post,
                    float* H_res, void* stream);
+
+/*
+ * mhc_phi_tf32_pair -- the projection matrix in tf32 ([mHC] section 4.3.1,
+ * Eq.(10): phi is tfloat32 while x is bfloat16) as an exact pair of bf16 rows,
+ * the phi operand of mhc_pre with phi_dt = MHC_TF32_PAIR.  Run once per update
+ * of phi.
+ *
+ * Every element of phi is first rounded to tf32 (10 explicit mantissa bits,
+ * round to nearest even; a no-op for values already in tf32), t; then
+ * hi = bf16(t) (round to nearest even) and lo = t - hi, which is a bf16 value,
+ * so hi + lo = t exactly for |t| >= 2^-116.
+ *
+ *   phi   [P][n*C] fp32, P = n*n + 2n: phi^T, as for mhc_pre (read)
+ *   pair  [2*RH][n*C] bf16, RH = P rounded up to a multiple of 16: rows
+ *         0..P-1 = hi, RH..RH+P-1 = lo, the other rows 0 (written;
+ *         mhc_phi_tf32_pair_bytes(n, C) bytes, must not overlap phi)
+ * 1 <= n <= 8, C a positive multiple of 8.
+ */
+size_t mhc_phi_tf32_pair_bytes(int n, int C);
+mhc_status mhc_phi_tf32_pair(const float* phi, int n, int C, void* pair, void* stream);
 
 /*
  * mhc_post -- the post half of one mHC sublayer.   [mHC] Eq.(3) and the fused

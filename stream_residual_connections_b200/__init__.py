@@ -22,7 +22,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmhc.so")
 
 MHC_OK, MHC_ERR_INVALID_ARG, MHC_ERR_UNSUPPORTED, MHC_ERR_CUDA, MHC_ERR_TIMEOUT = range(5)
-MHC_F32, MHC_BF16 = 0, 1
+MHC_F32, MHC_BF16, MHC_TF32_PAIR = 0, 1, 2
 MHC_PATH_AUTO, MHC_PATH_FMA, MHC_PATH_TENSOR = 0, 1, 2
 _STATUS = {0: "MHC_OK", 1: "MHC_ERR_INVALID_ARG", 2: "MHC_ERR_UNSUPPORTED", 3: "MHC_ERR_CUDA",
            4: "MHC_ERR_TIMEOUT"}
@@ -60,9 +60,12 @@ def _load():
     L.mhc_set_wait_limit.argtypes = [ct.c_longlong]
     L.hc_pre.argtypes = [vp, i32, vp, i32, fp, vp, i64, i32, i32, f32, vp, vp, vp, vp, vp]
     L.mhc_amax_gain.argtypes = [vp, i32, i64, i32, vp, vp, vp]
+    L.mhc_phi_tf32_pair.argtypes = [vp, i32, i32, vp, vp]
+    L.mhc_phi_tf32_pair_bytes.argtypes = [i32, i32]
+    L.mhc_phi_tf32_pair_bytes.restype = ct.c_size_t
     for name in ("mhc_pre", "mhc_post", "mhc_sync_status", "mhc_set_path", "mhc_set_wait_limit",
                  "xhc_conv_gs", "xhc_sparse_update", "xhc_route", "mhc_backward",
-                 "mhc_backward_noalloc", "hc_pre", "mhc_amax_gain"):
+                 "mhc_backward_noalloc", "hc_pre", "mhc_amax_gain", "mhc_phi_tf32_pair"):
         getattr(L, name).restype = ct.c_int
     return L
 
@@ -114,11 +117,27 @@ def _host3(alpha, count=3):
     return (ct.c_float * count)(*vals)
 
 
+def mhc_phi_tf32_pair(phi, n: int, *, pair=None, stream=None):
+    """The tf32 projection (the pages' Eq.10 dtype) as its exact bf16 pair, the phi
+    operand of mhc_pre(..., phi_tf32_pair=True).  phi: fp32 phi^T [n^2+2n][nC]; every
+    element is rounded to tf32 first.  Returns the pair [2*RH][nC] bf16."""
+    P, K = phi.shape
+    if phi.dtype != torch.float32 or P != n * n + 2 * n or K % n:
+        raise ValueError("phi must be fp32 [n^2+2n][n*C]")
+    C = K // n
+    RH = (P + 15) // 16 * 16
+    if pair is None:
+        pair = torch.empty((2 * RH, K), dtype=torch.bfloat16, device=phi.device)
+    _check(native().mhc_phi_tf32_pair(_ptr(phi), n, C, _ptr(pair), _stream(stream)))
+    return pair
+
+
 def mhc_pre(X, phi, alpha, b, t_iters: int = 20, eps: float = 1e-6, *, x_in=None, H_pre=None,
-            H_post=None, H_res=None, want_H_pre: bool = True, stream=None):
+            H_post=None, H_res=None, want_H_pre: bool = True, phi_tf32_pair: bool = False, stream=None):
     """Pre half of one mHC sublayer (see include/mhc.h).  X [T][n][C], phi [n^2+2n][nC]
-    (the projection stored transposed, like a linear layer's weight),
-    alpha: 3 host floats, b [n^2+2n] fp32.  Returns (x_in, H_pre, H_post, H_res)."""
+    (the projection stored transposed, like a linear layer's weight), or with
+    phi_tf32_pair=True the pair from mhc_phi_tf32_pair; alpha: 3 host floats,
+    b [n^2+2n] fp32.  Returns (x_in, H_pre, H_post, H_res)."""
     T, n, C = X.shape
     dev = X.device
     if x_in is None:
@@ -129,7 +148,8 @@ def mhc_pre(X, phi, alpha, b, t_iters: int = 20, eps: float = 1e-6, *, x_in=None
         H_post = torch.empty((T, n), dtype=torch.float32, device=dev)
     if H_res is None:
         H_res = torch.empty((T, n, n), dtype=torch.float32, device=dev)
-    _check(native().mhc_pre(_ptr(X), _dt(X), _ptr(phi), _dt(phi), _host3(alpha), _ptr(b), T, n, C,
+    pdt = MHC_TF32_PAIR if phi_tf32_pair else _dt(phi)
+    _check(native().mhc_pre(_ptr(X), _dt(X), _ptr(phi), pdt, _host3(alpha), _ptr(b), T, n, C,
                        int(t_iters), float(eps), _ptr(x_in), _ptr(H_pre), _ptr(H_post),
                        _ptr(H_res), _stream(stream)))
     return x_in, H_pre, H_post, H_res

@@ -81,7 +81,8 @@ mhc_status mhc_pre(const void* X, mhc_dtype x_dt, const void* phi, mhc_dtype phi
 {
     const char* fn = "mhc_pre";
     g_msg[0] = 0;
-    REQUIRE(valid_dt(x_dt) && valid_dt(phi_dt), MHC_ERR_INVALID_ARG, "%s: unknown dtype", fn);
+    const bool pair = phi_dt == MHC_TF32_PAIR;
+    REQUIRE(valid_dt(x_dt) && (valid_dt(phi_dt) || pair), MHC_ERR_INVALID_ARG, "%s: unknown dtype", fn);
     REQUIRE(n >= 1 && n <= 8, MHC_ERR_INVALID_ARG, "%s: n=%d outside [1, 8]", fn, n);
     REQUIRE(C > 0 && C % 8 == 0, MHC_ERR_INVALID_ARG, "%s: C=%d must be a positive multiple of 8", fn, C);
     REQUIRE(T >= 0, MHC_ERR_INVALID_ARG, "%s: T=%lld < 0", fn, (long long)T);
@@ -90,6 +91,7 @@ mhc_status mhc_pre(const void* X, mhc_dtype x_dt, const void* phi, mhc_dtype phi
     REQUIRE(alpha != nullptr, MHC_ERR_INVALID_ARG, "%s: alpha (host float[3]) is NULL", fn);
     REQUIRE(!(x_dt == MHC_F32 && phi_dt == MHC_BF16), MHC_ERR_UNSUPPORTED,
             "%s: fp32 X with bf16 phi is not supported", fn);
+    REQUIRE(!(x_dt == MHC_F32 && pair), MHC_ERR_UNSUPPORTED, "%s: the tf32 phi pair needs bf16 X", fn);
     if (T == 0) return MHC_OK;
     REQUIRE_PTR(X, "X");
     REQUIRE_PTR(phi, "phi");
@@ -100,7 +102,8 @@ mhc_status mhc_pre(const void* X, mhc_dtype x_dt, const void* phi, mhc_dtype phi
     if (H_pre) REQUIRE(aligned16(H_pre), MHC_ERR_INVALID_ARG, "%s: H_pre is not 16-byte aligned", fn);
     const int P = n * n + 2 * n;
     const size_t es = dt_size(x_dt);
-    const Range rX = range_of(X, size_t(T) * n * C * es), rphi = range_of(phi, size_t(n) * C * P * dt_size(phi_dt)),
+    const size_t phi_bytes = pair ? size_t(2 * tf32_pair_half_rows(n)) * n * C * 2 : size_t(n) * C * P * dt_size(phi_dt);
+    const Range rX = range_of(X, size_t(T) * n * C * es), rphi = range_of(phi, phi_bytes),
                 rb = range_of(b, size_t(P) * 4);
     const Range outs[4] = {range_of(x_in, size_t(T) * C * es), range_of(H_pre, H_pre ? size_t(T) * n * 4 : 0),
                            range_of(H_post, size_t(T) * n * 4), range_of(H_res, size_t(T) * n * n * 4)};
@@ -116,7 +119,8 @@ mhc_status mhc_pre(const void* X, mhc_dtype x_dt, const void* phi, mhc_dtype phi
     const bool tc_ok = pre_tc_supported(a), wide_ok = pre_wide_supported(a);
     if (g_pre_path == MHC_PATH_TENSOR && !tc_ok && !wide_ok) {
         set_error("%s: the tensor-core path was forced but does not support this call "
-                  "(needs bf16 X and phi, n in [2, 8], C %% 512 == 0)", fn);
+                  "(needs bf16 X, bf16 phi with n in [2, 8] or the tf32 phi pair with n <= 7, "
+                  "C %% 512 == 0)", fn);
         return MHC_ERR_UNSUPPORTED;
     }
     if (tc_ok && g_pre_path != MHC_PATH_FMA) return launch_pre_tc(a, s);
@@ -186,6 +190,26 @@ mhc_status hc_pre(const void* X, mhc_dtype x_dt, const void* theta, mhc_dtype th
     }
     HcArgs a{X, x_dt, theta, theta_dt, {alpha[0], alpha[1], alpha[2]}, b, T, n, C, eps, x_in, H_pre, H_post, H_res};
     return launch_hc_pre(a, static_cast<cudaStream_t>(stream));
+}
+
+size_t mhc_phi_tf32_pair_bytes(int n, int C)
+{
+    if (n < 1 || n > 8 || C <= 0) return 0;
+    return size_t(2 * tf32_pair_half_rows(n)) * n * C * 2;
+}
+
+mhc_status mhc_phi_tf32_pair(const float* phi, int n, int C, void* pair, void* stream)
+{
+    const char* fn = "mhc_phi_tf32_pair";
+    g_msg[0] = 0;
+    REQUIRE(n >= 1 && n <= 8, MHC_ERR_INVALID_ARG, "%s: n=%d outside [1, 8]", fn, n);
+    REQUIRE(C > 0 && C % 8 == 0, MHC_ERR_INVALID_ARG, "%s: C=%d must be a positive multiple of 8", fn, C);
+    REQUIRE_PTR(phi, "phi");
+    REQUIRE_PTR(pair, "pair");
+    const int P = n * n + 2 * n;
+    REQUIRE(!overlap(range_of(phi, size_t(P) * n * C * 4), range_of(pair, mhc_phi_tf32_pair_bytes(n, C))),
+            MHC_ERR_INVALID_ARG, "%s: pair overlaps phi", fn);
+    return launch_phi_tf32_pair(phi, n, C, pair, static_cast<cudaStream_t>(stream));
 }
 
 mhc_status mhc_amax_gain(const float* H_res, int L, int64_t T, int n, float* gain, float* gain_max, void* stream)

@@ -30,7 +30,7 @@ mhc_status launch_pre_fma(const PreArgs& a, cudaStream_t s);
 // {2, 3, 4}, C % 512 == 0 and phi's per-CTA slice resident in shared memory.
 bool pre_tc_supported(const PreArgs& a);
 mhc_status launch_pre_tc(const PreArgs& a, cudaStream_t s);
-bool pre_wide_supported(const PreArgs& a);                       // n = 5..8 (mhc_pre_wide.cu)
+bool pre_wide_supported(const PreArgs& a);   // bf16 phi, n = 5..8; tf32 pair phi, n = 1..7 (mhc_pre_wide.cu)
 mhc_status launch_pre_wide(const PreArgs& a, cudaStream_t s);
 
 mhc_status launch_conv_gs(const void* F, mhc_dtype dt, const float* W, const int* kappa, int r,
@@ -65,6 +65,10 @@ struct BwdArgs {
 int backward_b3_segments(int64_t T);
 size_t backward_record_stride(int n);            // floats per token record (0: unsupported n)
 mhc_status launch_backward(const BwdArgs& a, cudaStream_t s);
+
+// tf32 phi as an exact pair of bf16 rows (phi_tf32.cu): [2 RH][n C], RH = P rounded up to 16.
+inline int tf32_pair_half_rows(int n) { return (n * n + 2 * n + 15) / 16 * 16; }
+mhc_status launch_phi_tf32_pair(const float* phi, int n, int C, void* pair, cudaStream_t s);
 
 // HC (tanh) coefficients + F_pre input (hc_pre.cu); Amax Gain of a stack of H_res.
 struct HcArgs {

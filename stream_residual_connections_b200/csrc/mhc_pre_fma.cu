@@ -15,16 +15,39 @@
 // This path handles every n in [1, 8], both dtypes and any C % 8 == 0.  Its
 // projection costs 2 n C P flops per token on the FMA pipe, which for n >= 4
 // is more than the HBM time of the row; the tensor-core path is the fast one.
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace mhc {
 
-template <typename TP> struct PhiVec { static constexpr int W = 16 / sizeof(TP); };
+// phi storage: float, bf16, or the exact bf16 pair of a tf32 phi (phi_tf32.cu:
+// rows hi at p, lo at RH + p); PhiStore is the element type in memory.
+struct Tf32Pair {};
+template <typename TP> struct PhiStore { using type = TP; };
+template <> struct PhiStore<Tf32Pair> { using type = bf16_t; };
+template <typename TP> struct PhiVec { static constexpr int W = 16 / sizeof(typename PhiStore<TP>::type); };
+
+// Weights of logit p at columns k..k+W-1 of vec(X) (W = one 16-byte load).
+template <typename TP, int P>
+__device__ __forceinline__ void load_phi(const typename PhiStore<TP>::type* phiT, int p, int64_t K, int64_t k,
+                                         float (&pv)[PhiVec<TP>::W]) {
+    if constexpr (std::is_same<TP, Tf32Pair>::value) {
+        constexpr int RH = (P + 15) / 16 * 16;
+        float lo[PhiVec<TP>::W];
+        load16<false>(phiT + int64_t(p) * K + k, pv);
+        load16<false>(phiT + int64_t(RH + p) * K + k, lo);
+#pragma unroll
+        for (int e = 0; e < PhiVec<TP>::W; ++e) pv[e] += lo[e];      // exact: the pair sums to the tf32 value
+    } else {
+        load16<false>(phiT + int64_t(p) * K + k, pv);
+    }
+}
 
 template <int N, typename TX, typename TP>
 __global__ void __launch_bounds__(256)
-pre_fma_kernel(const TX* __restrict__ X, const TP* __restrict__ phiT, float a0, float a1, float a2,
+pre_fma_kernel(const TX* __restrict__ X, const typename PhiStore<TP>::type* __restrict__ phiT, float a0, float a1, float a2,
                const float* __restrict__ b, int64_t T, int C, int t_iters, float eps,
                TX* __restrict__ x_in, float* __restrict__ Hpre, float* __restrict__ Hpost,
                float* __restrict__ Hres, float* __restrict__ u_out, float* __restrict__ r_out)
@@ -53,7 +76,7 @@ pre_fma_kernel(const TX* __restrict__ X, const TP* __restrict__ phiT, float a0, 
 #pragma unroll
             for (int h = 0; h < W; h += PW) {
                 float pv[PW];
-                load16<false>(phiT + int64_t(p) * K + k0 + h, pv);
+                load_phi<TP, P>(phiT, p, K, k0 + h, pv);
 #pragma unroll
                 for (int e = 0; e < PW; ++e) acc[p] = fmaf(xv[h + e], pv[e], acc[p]);
             }
@@ -117,7 +140,7 @@ static mhc_status launch_pre_fma_n(const PreArgs& a, cudaStream_t s)
     const int warps = 8;
     const int64_t blocks = (a.T + warps - 1) / warps;
     pre_fma_kernel<N, TX, TP><<<dim3(unsigned(blocks)), warps * 32, 0, s>>>(
-        static_cast<const TX*>(a.X), static_cast<const TP*>(a.phi), a.alpha[0], a.alpha[1],
+        static_cast<const TX*>(a.X), static_cast<const typename PhiStore<TP>::type*>(a.phi), a.alpha[0], a.alpha[1],
         a.alpha[2], a.b, a.T, a.C, a.t_iters, a.eps, a.skip_xin ? nullptr : static_cast<TX*>(a.x_in),
         a.H_pre, a.H_post, a.H_res, a.u_out, a.r_out);
     return launch_status("mhc_pre (fma) kernel");
@@ -129,6 +152,7 @@ static mhc_status dispatch_dtype(const PreArgs& a, cudaStream_t s)
     if (a.x_dt == MHC_F32 && a.phi_dt == MHC_F32) return launch_pre_fma_n<N, float, float>(a, s);
     if (a.x_dt == MHC_BF16 && a.phi_dt == MHC_BF16) return launch_pre_fma_n<N, bf16_t, bf16_t>(a, s);
     if (a.x_dt == MHC_BF16 && a.phi_dt == MHC_F32) return launch_pre_fma_n<N, bf16_t, float>(a, s);
+    if (a.x_dt == MHC_BF16 && a.phi_dt == MHC_TF32_PAIR) return launch_pre_fma_n<N, bf16_t, Tf32Pair>(a, s);
     set_error("mhc_pre: dtype pair (x=%d, phi=%d) not supported", int(a.x_dt), int(a.phi_dt));
     return MHC_ERR_UNSUPPORTED;
 }

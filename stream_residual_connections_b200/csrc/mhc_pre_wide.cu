@@ -1,6 +1,8 @@
 // mhc_pre for n = 5..8 streams, tensor-core path: a projection kernel
 // (TMA + tcgen05.mma + TMEM, clusters of 8 CTAs) that writes the coefficients,
-// then a streaming x_in pass.
+// then a streaming x_in pass.  The same kernel serves every n <= 7 when phi is
+// given in tf32 ([mHC] Eq.(10)) as its exact bf16 pair (phi_tf32.cu): the stage
+// then carries both halves of phiT and the epilogue adds their columns.
 //
 // [mHC] section 4.3.1, Eq.(14)-(19), and F_pre := H_pre x_l, as in
 // mhc_pre_tc.cu.  With n >= 5 the projection has P = n^2 + 2n = 35..80
@@ -52,9 +54,12 @@ constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
 static_assert(TOK_PER_CTA * LPT == 64, "warps 2-3: one 4-lane group per token");
 
-template <int N> struct Cfg {
+// SPLIT: phi is the exact bf16 pair of a tf32 phi (phi_tf32.cu): the stage holds
+// hi rows [0, RH) and lo rows [RH, 2 RH), and logit p is column p + column RH + p.
+template <int N, bool SPLIT> struct Cfg {
     static constexpr int P = N * N + 2 * N;
-    static constexpr int R = (P + 15) / 16 * 16;   // phiT rows per stage (M = 128 needs N % 16 == 0)
+    static constexpr int RH = (P + 15) / 16 * 16;  // rows of one phiT half (M = 128 needs N % 16 == 0)
+    static constexpr int R = SPLIT ? 2 * RH : RH;  // phiT rows per stage
     static constexpr int MMA_N = R + MROWS;
     static constexpr int STAGE_BYTES = MMA_N * 128;
     static constexpr int PS = P + 1;
@@ -71,25 +76,25 @@ struct Layout {
     int stages;
 };
 
-template <int N>
+template <int N, bool SPLIT>
 __host__ __device__ constexpr uint32_t fixed_bytes() {
-    using G = Cfg<N>;
+    using G = Cfg<N, SPLIT>;
     return CL * TOK_PER_CTA * G::PSP * 4 + G::P * 4 + 16 + SINK_FLOATS * 4 + B_COUNT * 8 + 16;
 }
 
-template <int N>
+template <int N, bool SPLIT>
 __host__ __device__ constexpr int stages_fit() {
-    constexpr int64_t room = int64_t(SMEM_LIMIT) - 1024 - fixed_bytes<N>();
-    constexpr int64_t fit = room > 0 ? room / Cfg<N>::STAGE_BYTES : 0;
+    constexpr int64_t room = int64_t(SMEM_LIMIT) - 1024 - fixed_bytes<N, SPLIT>();
+    constexpr int64_t fit = room > 0 ? room / Cfg<N, SPLIT>::STAGE_BYTES : 0;
     return int(fit < MAX_STAGES ? fit : MAX_STAGES);
 }
 
-template <int N>
+template <int N, bool SPLIT>
 __host__ __device__ inline Layout layout_for() {
-    using G = Cfg<N>;
+    using G = Cfg<N, SPLIT>;
     Layout L;
     L.ring = 0;
-    L.stages = stages_fit<N>();
+    L.stages = stages_fit<N, SPLIT>();
     L.part = L.ring + uint32_t(L.stages) * G::STAGE_BYTES;
     L.bias = L.part + CL * TOK_PER_CTA * G::PSP * 4;
     L.sink = (L.bias + G::P * 4 + 15) / 16 * 16;
@@ -99,22 +104,22 @@ __host__ __device__ inline Layout layout_for() {
     return L;
 }
 
-template <int N>
+template <int N, bool SPLIT>
 __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NTHREADS, 1)
 proj_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmPhi, float a0,
             float a1, float a2, const float* __restrict__ b, int64_t T, int C, int Mt, int num_tiles, int t_iters,
             float eps, float* __restrict__ Hpre, float* __restrict__ Hpost, float* __restrict__ Hres,
             float* __restrict__ hpre_alt, int64_t alt_stride)
 {
-    using G = Cfg<N>;
-    constexpr int P = G::P, R = G::R, PS = G::PS, PSP = G::PSP, STAGE_BYTES = G::STAGE_BYTES;
+    using G = Cfg<N, SPLIT>;
+    constexpr int P = G::P, R = G::R, RH = G::RH, PS = G::PS, PSP = G::PSP, STAGE_BYTES = G::STAGE_BYTES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int Cs = C / CL;
     const int CB = Cs / KC;
     const int SPT = CB * N;            // ring stages per tile: (channel block, stream)
-    const Layout L = layout_for<N>();
+    const Layout L = layout_for<N, SPLIT>();
     const int STAGES = L.stages;
     uint8_t* sring = smem + L.ring;
     float* rpart = reinterpret_cast<float*>(smem + L.part);   // [CL][TOK_PER_CTA][PSP], pushed by the cluster
@@ -269,15 +274,21 @@ proj_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             }
             if (!warp_wait(&tfull[acc], uint32_t((it >> 1) & 1))) { s_abort = 1; alive = false; break; }
             tc_fence_after();
-            float d[R];
+            float d[RH];
             const uint32_t taddr = tmem_base + (uint32_t(qd * 32) << 16) + uint32_t(acc * ACC_COLS);
 #pragma unroll
-            for (int c = 0; c < R; c += 16) {
+            for (int c = 0; c < RH; c += 16) {
                 float tmp[16];
                 tmem_ld16(taddr + c, tmp);
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 16; ++j) d[c + j] = tmp[j];
+                if constexpr (SPLIT) {                  // x . lo, added to x . hi
+                    tmem_ld16(taddr + RH + c, tmp);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) d[c + j] += tmp[j];
+                }
             }
             float ss = 0.0f;
 #pragma unroll
@@ -405,12 +416,12 @@ xin_kernel(const bf16_t* __restrict__ X, const float* __restrict__ Hpre, int64_t
 
 // ------------------------------------------------------------------ host
 
-template <int N>
+template <int N, bool SPLIT>
 static mhc_status launch_n(const PreArgs& a, cudaStream_t s)
 {
     static int configured = 0, max_clusters = 0;
-    auto kern = proj_kernel<N>;
-    const int smem = int(layout_for<N>().total) + 1024;
+    auto kern = proj_kernel<N, SPLIT>;
+    const int smem = int(layout_for<N, SPLIT>().total) + 1024;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return cuda_status(e, "mhc_pre (n > 4): set shared memory size");
@@ -446,7 +457,7 @@ static mhc_status launch_n(const PreArgs& a, cudaStream_t s)
         set_error("mhc_pre (n > 4): cuTensorMapEncodeTiled unavailable");
         return MHC_ERR_CUDA;
     }
-    using G = Cfg<N>;
+    using G = Cfg<N, SPLIT>;
     CUtensorMap mapX, mapPhi;
     {
         // X [T][n][C] viewed as {C, T, n}: a box {64, Mt, 1} holds one stream's rows
@@ -463,8 +474,9 @@ static mhc_status launch_n(const PreArgs& a, cudaStream_t s)
         }
     }
     {
-        // phiT [P][n*C] viewed as {C, P, n}: a box {64, R, 1} holds R rows (rows >= P zero)
-        const cuuint64_t dims[3] = {cuuint64_t(a.C), cuuint64_t(G::P), cuuint64_t(N)};
+        // phiT [P][n*C] viewed as {C, P, n}: a box {64, R, 1} holds R rows (rows >= P
+        // zero); the tf32 pair [2 RH][n*C] as {C, 2 RH, n}: one box holds both halves
+        const cuuint64_t dims[3] = {cuuint64_t(a.C), cuuint64_t(SPLIT ? 2 * G::RH : G::P), cuuint64_t(N)};
         const cuuint64_t strides[2] = {cuuint64_t(N) * a.C * 2, cuuint64_t(a.C) * 2};
         const cuuint32_t box[3] = {KC, cuuint32_t(G::R), 1};
         const cuuint32_t estr[3] = {1, 1, 1};
@@ -494,17 +506,31 @@ static mhc_status launch_n(const PreArgs& a, cudaStream_t s)
 
 bool pre_wide_supported(const PreArgs& a)
 {
-    return a.x_dt == MHC_BF16 && a.phi_dt == MHC_BF16 && a.n >= 5 && a.n <= 8 && a.T >= 1 &&
-           a.T < (int64_t(1) << 31) && a.C % (prewide::CL * prewide::KC) == 0 && !a.skip_xin && !a.u_out;
+    const bool shape = (a.phi_dt == MHC_BF16 && a.n >= 5 && a.n <= 8) ||
+                       (a.phi_dt == MHC_TF32_PAIR && a.n >= 1 && a.n <= 7);   // 2 RH + 128 <= 256
+    return a.x_dt == MHC_BF16 && shape && a.T >= 1 && a.T < (int64_t(1) << 31) &&
+           a.C % (prewide::CL * prewide::KC) == 0 && !a.skip_xin && !a.u_out;
 }
 
 mhc_status launch_pre_wide(const PreArgs& a, cudaStream_t s)
 {
+    if (a.phi_dt == MHC_TF32_PAIR) {
+        switch (a.n) {
+            case 1: return prewide::launch_n<1, true>(a, s);
+            case 2: return prewide::launch_n<2, true>(a, s);
+            case 3: return prewide::launch_n<3, true>(a, s);
+            case 4: return prewide::launch_n<4, true>(a, s);
+            case 5: return prewide::launch_n<5, true>(a, s);
+            case 6: return prewide::launch_n<6, true>(a, s);
+            case 7: return prewide::launch_n<7, true>(a, s);
+            default: break;
+        }
+    }
     switch (a.n) {
-        case 5: return prewide::launch_n<5>(a, s);
-        case 6: return prewide::launch_n<6>(a, s);
-        case 7: return prewide::launch_n<7>(a, s);
-        case 8: return prewide::launch_n<8>(a, s);
+        case 5: return prewide::launch_n<5, false>(a, s);
+        case 6: return prewide::launch_n<6, false>(a, s);
+        case 7: return prewide::launch_n<7, false>(a, s);
+        case 8: return prewide::launch_n<8, false>(a, s);
         default: break;
     }
     set_error("mhc_pre (n > 4): n=%d not supported", a.n);

@@ -31,6 +31,17 @@ def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     return ((u + bias) >> 16).astype(np.uint16)
 
 
+def f32_to_tf32(a: np.ndarray) -> np.ndarray:
+    """Round float32 to tf32 (10 explicit mantissa bits, round-to-nearest-even on the
+    13 dropped bits); returns float32 values whose low 13 bits are zero."""
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    u = a.view(np.uint32)
+    finite = (u & np.uint32(0x7F800000)) != np.uint32(0x7F800000)
+    bias = ((u >> 13) & np.uint32(1)) + np.uint32(0xFFF)
+    r = np.where(finite, (u + bias) & np.uint32(0xFFFFE000), u)
+    return r.astype(np.uint32).view(np.float32)
+
+
 def _normal(rng: np.random.Generator, shape, std: float, dtype: str) -> np.ndarray:
     """float32 N(0, std^2) draws, stored as fp32 or as bf16 bits."""
     count = int(np.prod(shape)) if len(shape) else 1
@@ -46,20 +57,24 @@ def _normal(rng: np.random.Generator, shape, std: float, dtype: str) -> np.ndarr
 
 
 def mhc_inputs(T: int, n: int, C: int, dtype: str = "bf16", seed: int = 1,
-               alpha: float = 0.01) -> dict:
+               alpha: float = 0.01, phi_dtype: str | None = None) -> dict:
     """Inputs of one mHC sublayer (the mHC paper's Eq. 3 and Eq. 7-9 workload).
 
     Draw order: X ~ N(0,1) [T][n][C]; F_out ~ N(0,1) [T][C];
     phi ~ N(0, 1/(nC)) [nC][P]; b_pre ~ N(0, 0.1) [n]; b_post ~ N(0, 0.1) [n];
     the noise of b_res = 2*I_n + N(0, 0.1) [n][n].  X, F_out and phi take the
-    storage dtype; alpha (all three = ``alpha``) and b are float32.
+    storage dtype (phi_dtype="tf32": phi is the same float32 draw rounded to tf32
+    instead, stored as float32); alpha (all three = ``alpha``) and b are float32.
     """
-    assert dtype in ("bf16", "f32")
+    assert dtype in ("bf16", "f32") and phi_dtype in (None, "bf16", "f32", "tf32")
     P = n * n + 2 * n
     rng = np.random.Generator(np.random.PCG64(seed))
     X = _normal(rng, (T, n, C), 1.0, dtype)
     F = _normal(rng, (T, C), 1.0, dtype)
-    phi = _normal(rng, (n * C, P), float(1.0 / np.sqrt(n * C)), dtype)
+    pd = phi_dtype or dtype
+    phi = _normal(rng, (n * C, P), float(1.0 / np.sqrt(n * C)), "f32" if pd == "tf32" else pd)
+    if pd == "tf32":
+        phi = f32_to_tf32(phi)
     sd = float(np.sqrt(0.1))
     b_pre = rng.standard_normal(n, dtype=np.float32) * np.float32(sd)
     b_post = rng.standard_normal(n, dtype=np.float32) * np.float32(sd)
@@ -67,7 +82,7 @@ def mhc_inputs(T: int, n: int, C: int, dtype: str = "bf16", seed: int = 1,
              + np.float32(2.0) * np.eye(n, dtype=np.float32))
     b = np.concatenate([b_pre, b_post, b_res.reshape(-1)]).astype(np.float32)
     a = np.full(3, alpha, dtype=np.float32)
-    return dict(X=X, F=F, phi=phi, alpha=a, b=b, T=T, n=n, C=C, dtype=dtype,
+    return dict(X=X, F=F, phi=phi, alpha=a, b=b, T=T, n=n, C=C, dtype=dtype, phi_dtype=pd,
                 t_iters=20, eps=1e-6, seed=seed)
 
 
