@@ -288,8 +288,8 @@ mhc_status mhc_backward(const void* X, const void* F_out, const void* phi, mhc_d
  * workspace.  The scratch is a fixed MHC_NOALLOC_SCRATCH_BYTES (4 MiB) array
  * inside the library, held by every GPU that loads the library until the
  * process exits; batches whose mhc_backward_workspace_bytes(T, n, C) exceeds it
- * are rejected with MHC_ERR_UNSUPPORTED (at n = 4: T above about 5,200 at
- * C = 512, 2,000 at C = 2048, 1,000 at C = 4096).
+ * are rejected with MHC_ERR_UNSUPPORTED (at n = 4: T above about 4,600 at
+ * C = 512, 2,000 at C = 2048, 1,024 at C = 4096).
  * No allocating routine is called.  The first call on each device looks up
  * the scratch address and should come before any stream capture.  Every call
  * on a device uses the same scratch: calls whose work overlaps on the GPU

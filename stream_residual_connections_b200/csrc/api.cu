@@ -350,11 +350,13 @@ size_t mhc_backward_workspace_bytes(int64_t T, int n, int C)
     if (T < 0 || C < 0 || stride == 0) return 0;
     const size_t P = size_t(n) * n + 2 * n;
     const int segs = backward_b3_segments(T);
-    // per-token records, u and r; then the per-segment partial dphi sums
+    // per-token records, u and r; the dd^T bf16 pair of the tensor-core dphi product;
+    // then the per-segment partial dphi sums
     const size_t floats = size_t(T) * stride + size_t(T) * P + size_t(T);
     const size_t head = ((floats * 4 + 255) / 256) * 256;
+    const size_t ddt = ((size_t(64) * size_t(backward_ddt_pitch(T)) * 2 + 255) / 256) * 256;
     const size_t part = segs > 1 ? size_t(segs) * P * size_t(n) * size_t(C) * 4 : 0;
-    return head + part + 256;
+    return head + ddt + part + 256;
 }
 
 mhc_status mhc_backward(const void* X, const void* F_out, const void* phi, mhc_dtype dt, const float* alpha,
@@ -413,9 +415,10 @@ mhc_status mhc_backward(const void* X, const void* F_out, const void* phi, mhc_d
     float* ws = static_cast<float*>(workspace);
     const size_t stride = backward_record_stride(n);
     const size_t head_floats = (((size_t(T) * stride + size_t(T) * P + size_t(T)) * 4 + 255) / 256) * 256 / 4;
+    const size_t ddt_floats = ((size_t(64) * size_t(backward_ddt_pitch(T)) * 2 + 255) / 256) * 256 / 4;
     BwdArgs a{X, F_out, phi, dt, {alpha[0], alpha[1], alpha[2]}, b, dX_next, dx_in, T, n, C, t_iters, eps,
               dX, dF_out, dphi, dalpha, db, ws, ws + size_t(T) * stride, ws + size_t(T) * stride + size_t(T) * P,
-              ws + head_floats};
+              ws + head_floats + ddt_floats, ws + head_floats};
     return launch_backward(a, static_cast<cudaStream_t>(stream));
 }
 

@@ -61,8 +61,13 @@ struct BwdArgs {
     void* dX; void* dF; float* dphi; float* dalpha; float* db;
     float* records; float* u_scratch; float* r_scratch;   // carved from the caller's workspace
     float* dphi_part;                                     // [segments][P][nC] when segments > 1
+    void* ddt = nullptr;                                  // dd^T bf16 pair [64][pitch] (dphi on tensor cores)
 };
 int backward_b3_segments(int64_t T);
+inline int64_t backward_ddt_pitch(int64_t T) { return (T + 7) / 8 * 8; }   // 16-byte rows for TMA
+bool backward_dphi_tc_supported(const BwdArgs& a);
+mhc_status launch_backward_dphi_tc(const BwdArgs& a, int stride, int dd_off, int segs, int64_t seg_len,
+                                   cudaStream_t s);
 size_t backward_record_stride(int n);            // floats per token record (0: unsupported n)
 mhc_status launch_backward(const BwdArgs& a, cudaStream_t s);
 

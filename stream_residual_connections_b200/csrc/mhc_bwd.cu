@@ -511,9 +511,13 @@ static mhc_status run(const BwdArgs& a, cudaStream_t s)
     const int64_t K = int64_t(N) * a.C;
     const int segs = b3_segments(a.T);
     const int64_t seg_len = ((a.T + segs - 1) / segs + B3_T - 1) / B3_T * B3_T;
-    b3_kernel<N, TX><<<dim3(unsigned(K / B3_K), unsigned(segs)), 256, 0, s>>>(
-        static_cast<const TX*>(a.X), ws, a.T, a.C, seg_len, segs > 1 ? a.dphi_part : a.dphi);
-    st = launch_status("mhc_backward B3 kernel");
+    if (backward_dphi_tc_supported(a) && g_pre_path != MHC_PATH_FMA) {
+        st = launch_backward_dphi_tc(a, L::STRIDE, L::DD, segs, seg_len, s);     // tensor cores
+    } else {
+        b3_kernel<N, TX><<<dim3(unsigned(K / B3_K), unsigned(segs)), 256, 0, s>>>(
+            static_cast<const TX*>(a.X), ws, a.T, a.C, seg_len, segs > 1 ? a.dphi_part : a.dphi);
+        st = launch_status("mhc_backward B3 kernel");
+    }
     if (st != MHC_OK) return st;
     if (segs > 1) {
         const int64_t count = int64_t(P) * K;

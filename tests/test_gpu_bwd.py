@@ -69,6 +69,29 @@ def test_backward_matches_oracle(T, n, C, dtype):
     _compare(inp, _run(inp))
 
 
+@pytest.mark.parametrize("T,n,C", [(1500, 4, 256), (8200, 2, 128), (64, 1, 128), (77, 3, 512)])
+def test_backward_dphi_tensor_core_shapes(T, n, C):
+    """bf16 with nC % 128 == 0 takes the tensor-core dphi product (dd^T pair x X over
+    token segments): three segments with a ragged last one (T=1500), 16 segments of 576
+    tokens of which the last is empty and must contribute zeros (T=8200), n = 1 and 3."""
+    inp = synth.mhc_grad_inputs(T, n, C, "bf16", seed=830 + T + n + C)
+    _compare(inp, _run(inp))
+
+
+def test_backward_dphi_paths_agree():
+    """The tensor-core dphi product against the CUDA-core one on the same inputs."""
+    inp = synth.mhc_grad_inputs(1000, 4, 512, "bf16", seed=840)
+    try:
+        M.mhc_set_path(M.MHC_PATH_FMA)
+        a = _run(inp)
+    finally:
+        M.mhc_set_path(M.MHC_PATH_AUTO)
+    c = _run(inp)
+    scale = float(np.abs(a[2]).max())
+    assert np.abs(a[2] - c[2]).max() <= 1e-4 * scale
+    np.testing.assert_allclose(c[4], a[4], rtol=0, atol=1e-4 * float(np.abs(a[4]).max()))
+
+
 @pytest.mark.parametrize("t_iters", [0, 1, 5])
 def test_backward_short_sinkhorn(t_iters):
     inp = synth.mhc_grad_inputs(24, 4, 128, "f32", seed=810 + t_iters)
