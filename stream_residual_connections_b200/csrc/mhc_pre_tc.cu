@@ -78,9 +78,12 @@ constexpr int ACC_COLS = 256;             // TMEM columns per accumulator buffer
 constexpr int TMEM_COLS = 512;
 static_assert(TOK_PER_CTA * 8 == 64, "warps 4-5: one 8-lane group per coefficient token");
 
-template <int N> struct Cfg {
+// SPLIT: phi is the exact bf16 pair of a tf32 phi (phi_tf32.cu), rows hi [0, RH) and
+// lo [RH, 2 RH) per stream; a row's logit p is then column p + column RH + p of its half.
+template <int N, bool SPLIT = false> struct Cfg {
     static constexpr int P = N * N + 2 * N;
-    static constexpr int R = (P + 7) / 8 * 8;       // phiT rows per stream in a stage
+    static constexpr int RH = (P + 15) / 16 * 16;   // rows of one half of the tf32 pair
+    static constexpr int R = SPLIT ? 2 * RH : (P + 7) / 8 * 8;   // phiT rows per stream in a stage
     static constexpr int NP = (N + 1) / 2;          // stream pairs
     static constexpr int MMA_N = 2 * R + MROWS;     // B rows: the pair's phiT rows, then its X rows
     static constexpr int PAIR_BYTES = MMA_N * 128;
@@ -100,21 +103,21 @@ struct Layout {
 
 // Bytes after the ring: partial rows [CL][2 halves][TOK_PER_CTA][PSP], H_pre
 // [2][MT_CAP][N], b, barriers.
-template <int N>
+template <int N, bool SPLIT = false>
 __host__ __device__ constexpr uint32_t layout_fixed_bytes() {
-    using G = Cfg<N>;
+    using G = Cfg<N, SPLIT>;
     return CL * 2 * TOK_PER_CTA * G::PSP * 4 + 2 * MT_CAP * N * 4 + G::P * 4 + 16 + B_COUNT * 8 + 16;
 }
 
 // Shared memory plan: the ring takes as many stages (up to MAX_STAGES) as the
 // rest of the 227 KB leaves room for.
-template <int N>
+template <int N, bool SPLIT = false>
 __host__ __device__ inline Layout layout_for() {
-    using G = Cfg<N>;
+    using G = Cfg<N, SPLIT>;
     Layout L;
     L.ring = 0;
     {
-        const int64_t room = int64_t(SMEM_LIMIT) - 1024 - layout_fixed_bytes<N>();
+        const int64_t room = int64_t(SMEM_LIMIT) - 1024 - layout_fixed_bytes<N, SPLIT>();
         const int64_t fit = room > 0 ? room / G::STAGE_BYTES : 0;
         L.stages = int(fit < MAX_STAGES ? fit : MAX_STAGES);
     }
@@ -141,7 +144,7 @@ __device__ __forceinline__ void row_slot(int r, int Mt, int& h, int& tok) {
     }
 }
 
-template <int N>
+template <int N, bool SPLIT>
 __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(NTHREADS, 1)
 pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmPhi,
               const bf16_t* __restrict__ X, float a0, float a1, float a2,
@@ -150,7 +153,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
               float* __restrict__ Hpost, float* __restrict__ Hres, float* __restrict__ u_out,
               float* __restrict__ r_out)
 {
-    using G = Cfg<N>;
+    using G = Cfg<N, SPLIT>;
     constexpr int P = G::P, R = G::R, NP = G::NP, PS = G::PS, PSP = G::PSP;
     constexpr int STAGE_BYTES = G::STAGE_BYTES, PAIR_BYTES = G::PAIR_BYTES;
     extern __shared__ uint8_t smem_raw[];
@@ -159,7 +162,7 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
 
     const int Cs = C / CL;
     const int CB = Cs / KC;            // channel blocks = ring stages per tile
-    const Layout L = layout_for<N>();
+    const Layout L = layout_for<N, SPLIT>();
     const int STAGES = L.stages;
     uint8_t* sring = smem + L.ring;
     float* rpart = reinterpret_cast<float*>(smem + L.part);   // [CL][2][TOK_PER_CTA][PSP], pushed by the cluster
@@ -331,15 +334,29 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
             }
             if (!warp_wait(&tfull[acc], par)) { s_abort = 1; break; }
             tc_fence_after();
-            float d[2 * R];
+            // the row's projections: columns [h R, h R + P) of its half h (with the tf32
+            // pair, column h R + RH + q adds the lo part of logit q)
+            constexpr int DW = SPLIT ? G::RH : 2 * R;
+            float d[DW];
             const uint32_t taddr = tmem_base + (uint32_t(qd * 32) << 16) + uint32_t(acc * ACC_COLS);
+            if constexpr (SPLIT) {
+#pragma unroll
+                for (int q = 0; q < DW; ++q) d[q] = 0.0f;
+            }
 #pragma unroll
             for (int c = 0; c < 2 * R; c += 16) {
                 float tmp[16];
                 tmem_ld16(taddr + c, tmp);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) if (c + j < 2 * R) d[c + j] = tmp[j];
+                for (int j = 0; j < 16; ++j) {
+                    if constexpr (SPLIT) {
+                        const int col = c + j, hc = col / R, q = (col % R) % G::RH;   // compile-time
+                        if (hc == h) d[q] += tmp[j];
+                    } else {
+                        if (c + j < 2 * R) d[c + j] = tmp[j];
+                    }
+                }
             }
             float ss = 0.0f;
 #pragma unroll
@@ -364,7 +381,10 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int q = p + e;
-                    w[e] = q < P ? (h ? d[R + q] : d[q]) : (q == P ? ss : 0.0f);   // q < P <= R
+                    if constexpr (SPLIT)
+                        w[e] = q < P ? d[q] : (q == P ? ss : 0.0f);
+                    else
+                        w[e] = q < P ? (h ? d[R + q] : d[q]) : (q == P ? ss : 0.0f);   // q < P <= R
                 }
                 st_async_f32x4(push_dst + p * 4, make_float4(w[0], w[1], w[2], w[3]), push_bar);
             }
@@ -504,22 +524,22 @@ pre_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ C
 
 // ------------------------------------------------------------------ host
 
-template <int N>
-static int smem_bytes() { return int(layout_for<N>().total) + 1024; }
+template <int N, bool SPLIT>
+static int smem_bytes() { return int(layout_for<N, SPLIT>().total) + 1024; }
 
-template <int N>
+template <int N, bool SPLIT>
 static bool fits(int C)
 {
-    return C % (CL * KC) == 0 && layout_for<N>().stages >= 2 && smem_bytes<N>() <= SMEM_LIMIT;
+    return C % (CL * KC) == 0 && layout_for<N, SPLIT>().stages >= 2 && smem_bytes<N, SPLIT>() <= SMEM_LIMIT;
 }
 
-template <int N>
+template <int N, bool SPLIT>
 static mhc_status launch_n(const PreArgs& a, cudaStream_t s)
 {
     static int configured_smem = 0;
     static int max_clusters = 0;
-    const int smem = smem_bytes<N>();
-    auto kern = pre_tc_kernel<N>;
+    const int smem = smem_bytes<N, SPLIT>();
+    auto kern = pre_tc_kernel<N, SPLIT>;
     if (smem > configured_smem) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return cuda_status(e, "mhc_pre (tc): set shared memory size");
@@ -562,7 +582,7 @@ static mhc_status launch_n(const PreArgs& a, cudaStream_t s)
         set_error("mhc_pre (tc): cuTensorMapEncodeTiled unavailable");
         return MHC_ERR_CUDA;
     }
-    using G = Cfg<N>;
+    using G = Cfg<N, SPLIT>;
     CUtensorMap mapX, mapPhi;
     {
         // X [T][n][C] viewed as {C, T, n}: a box {64, Mt, 2} lands stream-major
@@ -581,8 +601,9 @@ static mhc_status launch_n(const PreArgs& a, cudaStream_t s)
     }
     {
         // phiT [P][n*C] viewed as {C, P, n}: a box {64, R, 2} holds the R rows
-        // (rows >= P zero-filled) of streams 2p and 2p+1 for one channel block
-        const cuuint64_t dims[3] = {cuuint64_t(a.C), cuuint64_t(G::P), cuuint64_t(a.n)};
+        // (rows >= P zero-filled) of streams 2p and 2p+1 for one channel block; the
+        // tf32 pair [2 RH][n*C] as {C, 2 RH, n}: both halves in the R = 2 RH rows
+        const cuuint64_t dims[3] = {cuuint64_t(a.C), cuuint64_t(SPLIT ? 2 * G::RH : G::P), cuuint64_t(a.n)};
         const cuuint64_t strides[2] = {cuuint64_t(a.n) * a.C * 2, cuuint64_t(a.C) * 2};
         const cuuint32_t box[3] = {KC, cuuint32_t(G::R), 2};
         const cuuint32_t estr[3] = {1, 1, 1};
@@ -605,21 +626,24 @@ static mhc_status launch_n(const PreArgs& a, cudaStream_t s)
 
 bool pre_tc_supported(const PreArgs& a)
 {
-    if (a.x_dt != MHC_BF16 || a.phi_dt != MHC_BF16 || a.T < 1 || a.T >= (int64_t(1) << 31)) return false;
+    const bool split = a.phi_dt == MHC_TF32_PAIR;
+    if (a.x_dt != MHC_BF16 || (a.phi_dt != MHC_BF16 && !split) || a.T < 1 || a.T >= (int64_t(1) << 31))
+        return false;
     switch (a.n) {
-        case 2: return pretc::fits<2>(a.C);
-        case 3: return pretc::fits<3>(a.C);
-        case 4: return pretc::fits<4>(a.C);
+        case 2: return split ? pretc::fits<2, true>(a.C) : pretc::fits<2, false>(a.C);
+        case 3: return split ? pretc::fits<3, true>(a.C) : pretc::fits<3, false>(a.C);
+        case 4: return split ? pretc::fits<4, true>(a.C) : pretc::fits<4, false>(a.C);
         default: return false;
     }
 }
 
 mhc_status launch_pre_tc(const PreArgs& a, cudaStream_t s)
 {
+    const bool split = a.phi_dt == MHC_TF32_PAIR;
     switch (a.n) {
-        case 2: return pretc::launch_n<2>(a, s);
-        case 3: return pretc::launch_n<3>(a, s);
-        case 4: return pretc::launch_n<4>(a, s);
+        case 2: return split ? pretc::launch_n<2, true>(a, s) : pretc::launch_n<2, false>(a, s);
+        case 3: return split ? pretc::launch_n<3, true>(a, s) : pretc::launch_n<3, false>(a, s);
+        case 4: return split ? pretc::launch_n<4, true>(a, s) : pretc::launch_n<4, false>(a, s);
         default: break;
     }
     set_error("mhc_pre (tc): n=%d not supported", a.n);
