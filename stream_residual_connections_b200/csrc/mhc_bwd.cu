@@ -509,10 +509,25 @@ static mhc_status run(const BwdArgs& a, cudaStream_t s)
     st = launch_status("mhc_backward B2 kernel");
     if (st != MHC_OK) return st;
     const int64_t K = int64_t(N) * a.C;
-    const int segs = b3_segments(a.T);
-    const int64_t seg_len = ((a.T + segs - 1) / segs + B3_T - 1) / B3_T * B3_T;
+    int segs = b3_segments(a.T);
+    int64_t seg_len = ((a.T + segs - 1) / segs + B3_T - 1) / B3_T * B3_T;
     if (backward_dphi_tc_supported(a) && g_pre_path != MHC_PATH_FMA) {
-        st = launch_backward_dphi_tc(a, L::STRIDE, L::DD, segs, seg_len, s);     // tensor cores
+        // tensor cores: long token segments (a CTA's fixed costs -- TMEM, ring fill,
+        // epilogue -- against its streaming), about two CTAs per SM in one wave; at most
+        // the segments the workspace holds partials for
+        static int sms = 0;
+        if (!sms) {
+            int dev = 0;
+            cudaError_t e = cudaGetDevice(&dev);
+            if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess) return cuda_status(e, "mhc_backward: SM count");
+        }
+        const int64_t slabs = K / 128;
+        const int64_t want = (2 * int64_t(sms) + slabs / 2) / slabs;
+        const int segs_tc = int(want < 1 ? 1 : (want > segs ? segs : want));
+        segs = segs_tc;
+        seg_len = ((a.T + segs - 1) / segs + B3_T - 1) / B3_T * B3_T;
+        st = launch_backward_dphi_tc(a, L::STRIDE, L::DD, segs, seg_len, s);
     } else {
         b3_kernel<N, TX><<<dim3(unsigned(K / B3_K), unsigned(segs)), 256, 0, s>>>(
             static_cast<const TX*>(a.X), ws, a.T, a.C, seg_len, segs > 1 ? a.dphi_part : a.dphi);
