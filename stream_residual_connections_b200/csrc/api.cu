@@ -220,19 +220,23 @@ mhc_status mhc_amax_gain(const float* H_res, int L, int64_t T, int n, float* gai
     REQUIRE(L >= 0 && T >= 0, MHC_ERR_INVALID_ARG, "%s: L=%d, T=%lld must be >= 0", fn, L, (long long)T);
     REQUIRE(gain || gain_max, MHC_ERR_INVALID_ARG, "%s: neither gain nor gain_max given", fn);
     if (L == 0) return MHC_OK;
+    // every argument is checked before anything is enqueued
     if (gain_max) REQUIRE(aligned16(gain_max), MHC_ERR_INVALID_ARG, "%s: gain_max is not 16-byte aligned", fn);
+    if (T > 0) {
+        REQUIRE_PTR(H_res, "H_res");
+        if (gain) REQUIRE(aligned16(gain), MHC_ERR_INVALID_ARG, "%s: gain is not 16-byte aligned", fn);
+        const Range rH = range_of(H_res, size_t(L) * T * n * n * 4);
+        const Range rg = range_of(gain, gain ? size_t(L) * T * 2 * 4 : 0),
+                    rm = range_of(gain_max, gain_max ? size_t(L) * 8 : 0);
+        REQUIRE(!overlap(rg, rH) && !overlap(rm, rH) && !overlap(rg, rm), MHC_ERR_INVALID_ARG,
+                "%s: an output overlaps H_res or the other output", fn);
+    }
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (gain_max) {
         const mhc_status st = cuda_status(cudaMemsetAsync(gain_max, 0, size_t(L) * 2 * 4, s), fn);
         if (st != MHC_OK) return st;
     }
     if (T == 0) return MHC_OK;
-    REQUIRE_PTR(H_res, "H_res");
-    if (gain) REQUIRE(aligned16(gain), MHC_ERR_INVALID_ARG, "%s: gain is not 16-byte aligned", fn);
-    const Range rH = range_of(H_res, size_t(L) * T * n * n * 4);
-    const Range rg = range_of(gain, gain ? size_t(L) * T * 2 * 4 : 0), rm = range_of(gain_max, gain_max ? size_t(L) * 8 : 0);
-    REQUIRE(!overlap(rg, rH) && !overlap(rm, rH) && !overlap(rg, rm), MHC_ERR_INVALID_ARG,
-            "%s: an output overlaps H_res or the other output", fn);
     return launch_amax_gain(H_res, L, T, n, gain, gain_max, s);
 }
 
