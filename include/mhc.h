@@ -313,12 +313,15 @@ typedef enum {
 
 /*
  * mhc_set_path -- process-wide choice of the projection kernel of mhc_pre,
- * xhc_route and xhc_sparse_update (for comparisons and tests; both paths
- * compute the same function).  The tensor-core paths (TMA + tcgen05.mma, 8-CTA
- * clusters) serve bf16 X and phi, C % 512 == 0, 1 <= T < 2^31, and n in
- * {2, 3, 4} (mhc_pre), N in {4, 8, 12, 16} (xhc_route), k = 4 with Kr <= 4
- * (xhc_sparse_update).  Under MHC_PATH_TENSOR a call outside that range
- * returns MHC_ERR_UNSUPPORTED.
+ * xhc_route and xhc_sparse_update, and of the dphi product of mhc_backward
+ * (for comparisons and tests; both paths compute the same function).  The
+ * tensor-core paths (TMA + tcgen05.mma) serve bf16 X, 1 <= T < 2^31, and:
+ * mhc_pre with bf16 phi, C % 512 == 0 and n in [2, 8], or with the tf32 phi
+ * pair and n in [1, 7]; xhc_route with C % 512 == 0 and N in {4, 8, 12, 16};
+ * xhc_sparse_update with C % 512 == 0, k = 4 and Kr <= 4; mhc_backward's dphi
+ * with n*C % 128 == 0.  Under MHC_PATH_TENSOR an mhc_pre, xhc_route or
+ * xhc_sparse_update call outside that range returns MHC_ERR_UNSUPPORTED;
+ * MHC_PATH_FMA selects the CUDA-core kernels everywhere.
  */
 mhc_status mhc_set_path(mhc_path path);
 
