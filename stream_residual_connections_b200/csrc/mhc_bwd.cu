@@ -260,7 +260,7 @@ b1_kernel(const TX* __restrict__ X, const TX* __restrict__ F, const TX* __restri
 constexpr int B2_T = 64, B2_C = 64, B2_SUB = 16;   // tokens per block; per pass of the 128 threads
 
 template <int N, typename TX>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, 5)
 b2_kernel(const TX* __restrict__ X, const TX* __restrict__ dXn, const TX* __restrict__ dxin,
           const TX* __restrict__ phiT, const float* __restrict__ ws, int64_t T, int C, TX* __restrict__ dX)
 {
