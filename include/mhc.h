@@ -43,7 +43,7 @@ extern "C" {
 typedef enum {
     MHC_OK = 0,
     MHC_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, forbidden aliasing */
-    MHC_ERR_UNSUPPORTED = 2,  /* valid but outside what this build implements        */
+    MHC_ERR_UNSUPPORTED = 2,  /* valid but outside what this library implements      */
     MHC_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed                  */
     MHC_ERR_TIMEOUT = 4       /* a bounded on-device wait expired (see mhc_sync_status)*/
 } mhc_status;
@@ -243,7 +243,7 @@ mhc_status xhc_conv_gs(const void* F_out, mhc_dtype dt, const float* conv_w, con
  *           (row p = weights of logit p over vec(X_act)); rows res | post (read)
  *   alpha_act HOST float[2] = (alpha_res, alpha_post);  b_act [k*k + k*Kr] fp32
  *   H_res   [T][k][k] fp32, may be NULL;  H_post [T][k][Kr] fp32, may be NULL (written)
- * This build: k <= 4, Kr <= 5, C % 64 == 0, N <= 64.
+ * This library: k <= 4, Kr <= 5, C % 64 == 0, N <= 64.
  */
 mhc_status xhc_sparse_update(void* X, mhc_dtype dt, const float* V, int Kr, const int32_t* idx,
                              const float* w, const void* phi_act, const float* alpha_act,
@@ -268,7 +268,7 @@ mhc_status xhc_sparse_update(void* X, mhc_dtype dt, const float* V, int Kr, cons
  *   workspace: device scratch of at least mhc_backward_workspace_bytes(T, n, C)
  *   bytes, 256-byte aligned, owned by the caller; its contents on entry are
  *   ignored and on exit undefined.
- * This build: n <= 4, C % 64 == 0, t_iters <= 100.  T == 0 zeroes the sums.
+ * This library: n <= 4, C % 64 == 0, t_iters <= 100.  T == 0 zeroes the sums.
  */
 size_t mhc_backward_workspace_bytes(int64_t T, int n, int C);
 mhc_status mhc_backward(const void* X, const void* F_out, const void* phi, mhc_dtype dt,

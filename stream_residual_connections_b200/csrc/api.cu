@@ -320,7 +320,7 @@ mhc_status xhc_sparse_update(void* X, mhc_dtype dt, const float* V, int Kr, cons
     REQUIRE(t_iters >= 0 && t_iters <= 1000, MHC_ERR_INVALID_ARG, "%s: t_iters=%d outside [0, 1000]", fn, t_iters);
     REQUIRE(eps >= 0.0f, MHC_ERR_INVALID_ARG, "%s: eps < 0", fn);
     REQUIRE(alpha_act != nullptr, MHC_ERR_INVALID_ARG, "%s: alpha_act (host float[2]) is NULL", fn);
-    REQUIRE(k <= 4 && Kr <= 5, MHC_ERR_UNSUPPORTED, "%s: k=%d, Kr=%d (this build: k <= 4, Kr <= 5)", fn, k, Kr);
+    REQUIRE(k <= 4 && Kr <= 5, MHC_ERR_UNSUPPORTED, "%s: k=%d, Kr=%d (this library: k <= 4, Kr <= 5)", fn, k, Kr);
     REQUIRE(C % 64 == 0, MHC_ERR_UNSUPPORTED, "%s: C=%d must be a multiple of 64", fn, C);
     if (T == 0) return MHC_OK;
     REQUIRE_PTR(X, "X");
@@ -378,7 +378,7 @@ mhc_status mhc_backward(const void* X, const void* F_out, const void* phi, mhc_d
     REQUIRE(eps >= 0.0f, MHC_ERR_INVALID_ARG, "%s: eps < 0", fn);
     REQUIRE(alpha != nullptr, MHC_ERR_INVALID_ARG, "%s: alpha (host float[3]) is NULL", fn);
     REQUIRE(n <= 4 && C % 64 == 0 && t_iters <= 100, MHC_ERR_UNSUPPORTED,
-            "%s: this build needs n <= 4, C %% 64 == 0, t_iters <= 100", fn);
+            "%s: this library needs n <= 4, C %% 64 == 0, t_iters <= 100", fn);
     const int P = n * n + 2 * n;
     REQUIRE_PTR(dphi, "dphi");
     REQUIRE(dalpha != nullptr && db != nullptr, MHC_ERR_INVALID_ARG, "%s: dalpha or db is NULL", fn);
