@@ -71,7 +71,7 @@ constexpr int B1_THREADS = MHC_B1_THREADS;   // small blocks: the per-token seri
 constexpr int B1_WARPS = B1_THREADS / 32;    // several blocks overlap on an SM
 
 template <int N, typename TX>
-__global__ void __launch_bounds__(B1_THREADS)
+__global__ void __launch_bounds__(B1_THREADS, 5)
 b1_kernel(const TX* __restrict__ X, const TX* __restrict__ F, const TX* __restrict__ dXn,
           const TX* __restrict__ dxin, float a0, float a1, float a2, const float* __restrict__ b,
           int64_t T, int C, int t_iters, const float* __restrict__ uu, const float* __restrict__ rr,
